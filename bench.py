@@ -1,0 +1,540 @@
+#!/usr/bin/env python3
+"""Benchmark: NVFP4 paged decode step (quantize-append + paged attention).
+
+Workload: the Qwen3-0.6B-shaped decode batch (16 q / 8 kv heads, head_size
+128, block_size 16, 32 sequences with 512-4096 keys, N(0,1) K/V with 2% of
+(head, channel) pairs x20, random block tables). One step appends each
+sequence's new token (the quantize-append writer, 32 tokens) and runs decode
+attention over every sequence's keys (FP8 output + bf16 dequant).
+
+Timed region: W warm-up steps, then exactly K steps replayed from CUDA graphs,
+bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
+events on the launching stream, max over ranks. Inputs are rotated over
+enough independent copies (cache, tables, queries) to exceed 4x the 126 MB L2,
+so every step reads its KV from HBM.
+
+value = algorithmic NVFP4 KV bytes read per step (sum over sequences of
+seq_len * kv_heads * 2 * full_dim, no block padding) / step time, summed over
+ranks (each rank runs its own replica: the path has no exchange step).
+
+Also reported: roofline of the attention kernel (its own CUDA-event time per
+launch), the quantize-append sweep (8192 tokens into a 65536 x 16 cache) in
+Mtok/s, the end-to-end number through host buffers, the CPU oracle baseline
+and SM clocks sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 paged decode attn KV GB/s (% of HBM peak); append Mtok/s"
+WORKLOAD = "qwen3_0p6b_decode"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+def dist_init(n):
+    import torch
+    import torch.distributed as dist
+    if n <= 1 or "RANK" not in os.environ:
+        return 0, 1, None
+    from datetime import timedelta
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, dist.get_world_size(), dist
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(x, dist):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi SM clock + throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, time.time())
+        rows = [s for t, s in self.samples if t0 - 0.15 <= t <= t1 + 0.15] or \
+               [s for _, s in self.samples[-5:]]
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ our arm
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_quantized_paged_append_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class DecodeState:
+    """One independent copy of the step's device state."""
+
+    def __init__(self, w, scales, hist_cache, device):
+        import torch
+        import nvfp4_quantized_paged_append_b200 as nk
+        from nvfp4_quantized_paged_append_b200 import workloads as wl
+        self.cache = hist_cache.clone()
+        self.bt = torch.from_numpy(w.block_table).to(device)
+        self.sl = torch.from_numpy(w.seq_lens).to(device)
+        self.q = wl.queries(w, device)
+        B, H, D = w.num_seqs, w.num_kv_heads, w.head_size
+        # the new token of each sequence = its last position
+        ks, vs = [], []
+        for b in range(B):
+            k, v = wl.seq_kv(w, b, device, start=int(w.seq_lens[b]) - 1)
+            ks.append(k)
+            vs.append(v)
+        self.k_new = torch.cat(ks).contiguous()
+        self.v_new = torch.cat(vs).contiguous()
+        self.slots = torch.from_numpy(np.array(
+            [w.slots_for_seq(b, int(w.seq_lens[b]) - 1)[0] for b in range(B)], np.int64)).to(device)
+        self.kvs = torch.tensor([scales[0], scales[1]], dtype=torch.float32, device=device)
+        self.ks = self.kvs[0:1]
+        self.vs = self.kvs[1:2]
+        self.osc = torch.tensor([scales[2]], dtype=torch.float32, device=device)
+        self.o8 = torch.empty((B, w.num_q_heads, D), dtype=torch.uint8, device=device)
+        self.o16 = torch.empty((B, w.num_q_heads, D), dtype=torch.bfloat16, device=device)
+        self.ws = nk.alloc_workspace(B, w.num_q_heads, H, D, device)
+
+    def append(self, nk, stream=None):
+        nk.quantize_append_paged(self.k_new, self.v_new, self.cache, self.slots, self.ks, self.vs,
+                                 stream=stream)
+
+    def attend(self, nk, stream=None):
+        nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
+                           self.ws, o_bf16=self.o16, stream=stream)
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    nk.lib()
+
+    w = wl.make_workload(WORKLOAD)
+    scales = wl.global_scales(w, dev)
+    kv_bytes = w.kv_bytes()
+    # history: every token but the last, written once by the library's writer
+    hist = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+    ksd = torch.tensor([scales[0]], dtype=torch.float32, device=dev)
+    vsd = torch.tensor([scales[1]], dtype=torch.float32, device=dev)
+    for b in range(w.num_seqs):
+        L = int(w.seq_lens[b])
+        k, v = wl.seq_kv(w, b, dev, stop=L - 1)
+        nk.quantize_append_paged(k, v, hist, torch.from_numpy(w.slots_for_seq(b, 0, L - 1)).to(dev),
+                                 ksd, vsd)
+    cache_bytes = hist.numel()
+    copies = max(2, -(-4 * L2_BYTES // cache_bytes) + 1)
+    states = [DecodeState(w, scales, hist, dev) for _ in range(copies)]
+    del hist
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    for st in states:  # eager run of every copy before capture (first calls are eager)
+        st.append(nk, stream)
+        st.attend(nk, stream)
+    stream.synchronize()
+    # NG graphs of R = copies steps each; every attention launch in them is
+    # bracketed by its own external (graph-node) timing events, so the kernel's
+    # own device time is measured inside the timed region itself. One-step
+    # graphs serve the K mod R remainder.
+    NG = 4
+    group_graphs, group_events = [], []
+    for g in range(NG):
+        graph = torch.cuda.CUDAGraph()
+        evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(copies)]
+        with torch.cuda.graph(graph, stream=stream):
+            for i, st in enumerate(states):
+                st.append(nk, stream)
+                evs[i][0].record(stream)
+                st.attend(nk, stream)
+                evs[i][1].record(stream)
+        group_graphs.append(graph)
+        group_events.append(evs)
+    single = []
+    for st in states:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            st.append(nk, stream)
+            st.attend(nk, stream)
+        single.append(graph)
+
+    def run_steps(n):
+        full, rem = divmod(n, copies)
+        for j in range(full):
+            group_graphs[j % NG].replay()
+        for j in range(rem):
+            single[j].replay()
+        return min(full, NG)
+
+    run_steps(max(3, args.warmup))
+    stream.synchronize()
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    # keep the GPU under the same load ~1.5 s before the timed region so the
+    # sampled clocks are the loaded ones (extra warm-up, not timed)
+    t_end = time.time() + 1.5
+    while time.time() < t_end:
+        run_steps(NG * copies * 8)
+        stream.synchronize()
+    barrier(dist)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark()
+    e0.record(stream)
+    used_groups = run_steps(args.steps)
+    e1.record(stream)
+    stream.synchronize()
+    clocks.mark()
+    torch.cuda.synchronize()
+    barrier(dist)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, dist)
+    ms_step = ms / args.steps
+    clocks.stop()
+    # attention kernel durations from the last replay of each group graph
+    kt = [a.elapsed_time(b) for evs in group_events[:used_groups] for a, b in evs]
+    if not kt:  # fewer steps than one group: time one group replay now
+        group_graphs[0].replay()
+        stream.synchronize()
+        kt = [a.elapsed_time(b) for a, b in group_events[0]]
+    attn_ms = statistics.mean(kt)
+
+    # ---- quantize-append sweep (8192 tokens) for Mtok/s
+    app = wl.make_append()
+    ka, va = app.kv(dev)
+    gka, gva = app.scales(ka, va)
+    slots = torch.from_numpy(app.slot_mapping()).to(dev)
+    acache = nk.alloc_kv_cache(app.num_blocks, app.block_size, app.num_kv_heads, app.head_size, dev)
+    ksa = torch.tensor([gka], dtype=torch.float32, device=dev)
+    vsa = torch.tensor([gva], dtype=torch.float32, device=dev)
+    # rotate input copies so reads come from HBM (each copy ~32 MB of bf16)
+    acopies = max(2, -(-4 * L2_BYTES // (ka.numel() * 4)) + 1)
+    kas = [ka.clone() for _ in range(acopies)]
+    vas = [va.clone() for _ in range(acopies)]
+    nrep = 400
+    if True:
+        for i in range(20):
+            nk.quantize_append_paged(kas[i % acopies], vas[i % acopies], acache, slots, ksa, vsa,
+                                     stream=stream)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(nrep):
+            nk.quantize_append_paged(kas[i % acopies], vas[i % acopies], acache, slots, ksa, vsa,
+                                     stream=stream)
+        a1.record(stream)
+    stream.synchronize()
+    app_ms = a0.elapsed_time(a1) / nrep
+    app_bytes = app.algorithmic_bytes()
+
+    # ---- end to end through host buffers (pinned), every step: H2D of q, new k/v,
+    # slots, seq_lens, block table; D2H of the bf16 output
+    st = states[0]
+    host_in = {name: getattr(st, name).cpu().pin_memory()
+               for name in ("q", "k_new", "v_new", "slots", "sl", "bt")}
+    host_out = torch.empty_like(st.o16, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(50, min(500, args.steps))
+    if True:
+        for it in range(e2e_steps + 10):
+            if it == 10:
+                barrier(dist)
+                stream.synchronize()
+                x0 = torch.cuda.Event(enable_timing=True)
+                x0.record(stream)
+            stt = states[it % copies]
+            for name, t in host_in.items():
+                getattr(stt, name).copy_(t, non_blocking=True)
+            stt.append(nk, stream)
+            stt.attend(nk, stream)
+            host_out.copy_(stt.o16, non_blocking=True)
+        x1 = torch.cuda.Event(enable_timing=True)
+        x1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / e2e_steps, dist)
+
+    peak, peak_kind = peaks()
+    achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
+    traffic = profiled_traffic("decode_attention_kernel<128,16>@" + WORKLOAD)
+    result = {
+        "metric": METRIC,
+        "value": round(world * kv_bytes / (ms_step * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1+e4m3) kv, bf16 q, f16 mma, fp32 accum, e4m3 out",
+        "data": "synthetic (seeded N(0,1) K/V/Q, 2% outlier channels x20)",
+        "config": {
+            "workload": WORKLOAD, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_size": w.head_size,
+            "block_size": w.block_size, "ctx_lens": "uniform 512-4096 (seeded)",
+            "kv_bytes_per_step": kv_bytes, "new_tokens_per_step": w.num_seqs,
+            "l2": f"inputs rotated over {copies} copies ({copies * cache_bytes / 2**20:.0f} MiB of cache) > 4x L2",
+            "parallelism": f"replicas x{world} (independent shards, no collective)",
+            "step": "quantize-append of 32 new tokens + decode attention (CUDA graph replay)",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "decode_attention_kernel<128,16>",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} HBM copy",
+            "traffic": traffic, "algorithmic_bytes_per_launch": kv_bytes,
+            "kernel_ms": round(attn_ms, 5),
+            "frac_of_8TBps": round(achieved / 8000.0, 4),
+        },
+        "append": {
+            "workload": "append_sweep", "tokens": app.num_tokens, "live_tokens": app.live_tokens(),
+            "ms": round(app_ms, 5), "mtok_s": round(app.num_tokens / (app_ms * 1e-3) / 1e6, 1),
+            "gbs": round(app_bytes / (app_ms * 1e-3) / 1e9, 1),
+            "frac": round(app_bytes / (app_ms * 1e-3) / 1e9 / peak, 4),
+            "algorithmic_bytes": app_bytes,
+        },
+        "e2e": {
+            "value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(e2e_ms, 5),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        },
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    return result
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample_gbs(w, seqs, scales, budget_s=15.0):
+    """Time the CPU oracle on a bounded sample of the workload; KV GB/s."""
+    import torch
+    import oracle
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    q = u16(wl.queries(w, "cpu"))
+    blocks = {}
+    for b in seqs:
+        for x in w.block_table[b, : -(-int(w.seq_lens[b]) // w.block_size)]:
+            blocks.setdefault(int(x), len(blocks))
+    cache = np.zeros((len(blocks), 2, w.num_kv_heads, w.block_size, w.full_dim), np.uint8)
+    bt = np.zeros((len(seqs), w.max_blocks_per_seq), np.int32)
+    for i, b in enumerate(seqs):
+        L = int(w.seq_lens[b])
+        k, v = wl.seq_kv(w, b, "cpu")
+        n = np.arange(L)
+        loc = np.array([blocks[int(x)] for x in w.block_table[b, n // w.block_size]], np.int64)
+        oracle.quantize_append_paged(u16(k), u16(v), cache, loc * w.block_size + n % w.block_size,
+                                     scales[0], scales[1], w.block_size)
+        nblk = -(-L // w.block_size)
+        bt[i, :nblk] = [blocks[int(x)] for x in w.block_table[b, :nblk]]
+    sl = np.array([w.seq_lens[b] for b in seqs], np.int32)
+    qs = np.ascontiguousarray(q[list(seqs)])
+    kvb = int(sl.astype(np.int64).sum()) * w.num_kv_heads * 2 * w.full_dim
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.paged_attention(qs, cache, bt, sl, None, scales[0], scales[1], 0.0, scales[2])
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 50:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return kvb / dt / 1e9, dt, kvb
+
+
+def cpu_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    """The oracle (CPU, as it stands) on the same workload and metric."""
+    if rank != 0:
+        return None
+    import oracle
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    oracle.build()
+    w = wl.make_workload(WORKLOAD)
+    scales = wl.global_scales(w, "cpu")
+    seqs = [0, 1]
+    sample = f"oracle attention on sequences {seqs} of {w.num_seqs} per step"
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_gbs(w, seqs, scales, budget_s=0.0)
+    total_t, total_b = 0.0, 0
+    for _ in range(max(1, min(args.steps, 5))):
+        gbs, dt, kvb = oracle_sample_gbs(w, seqs, scales, budget_s=0.0)
+        total_t += dt
+        total_b += kvb
+    value = total_b / total_t / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": max(1, min(args.steps, 5)), "warmup": args.warmup,
+        "ms_per_step": round(total_t / max(1, min(args.steps, 5)) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, dist = dist_init(args.gpus)
+    res = run_ours(args, rank, world, dist)
+    if rank == 0 and not args.no_cpu_baseline:
+        # bounded CPU oracle sample (rank 0, 1 GPU only)
+        if world == 1:
+            from nvfp4_quantized_paged_append_b200 import workloads as wl
+            import oracle
+            oracle.build()
+            w = wl.make_workload(WORKLOAD)
+            scales = wl.global_scales(w, "cpu")
+            gbs, dt, kvb = oracle_sample_gbs(w, [0, 1], scales, budget_s=10.0)
+            res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(),
+                                   "kind": "oracle",
+                                   "sample": f"oracle attention, sequences 0-1 of {w.num_seqs} "
+                                             f"({kvb} KV bytes), repeated for ~10 s"}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * nvfp4kv -- NVFP4 paged KV cache for B200 (sm_100a): C ABI.
+ *
+ * Two hot operations and two helpers, after the pages on NVFP4 KV caches:
+ *   - "FlashInfer backend adds end-to-end NVFP4 KV cache support" (vLLM PR
+ *     #40177 summary), key source snippets: get_kv_cache_shape gives the
+ *     cache shape (num_blocks, 2, block_size, num_kv_heads, full_dim) with
+ *     full_dim = head_size/2 + head_size/16; _create_nvfp4_hnd_kv_cache stores
+ *     it in HND order (num_blocks, 2, num_kv_heads, block_size, full_dim) and
+ *     fills it with reshape_and_cache_flash(k, v, ..., slot_mapping, "nvfp4",
+ *     k_scale, v_scale); implementation breakdown items 2-3: the attention
+ *     kernel reads the packed data plus the FP8 block scales and writes FP8
+ *     output that is dequantized back to the model dtype.
+ *   - "FlashInfer NVFP4 KV serving on pre-SM100 GPUs" (vLLM RFC #47684),
+ *     quick answer: the slot-mapped NVFP4 append helper and the paged NVFP4
+ *     dequantize helper.
+ *   - "Move NVFP4 GEMM management into NvFp4LinearKernel" (vLLM PR #39129),
+ *     base.py, NvFp4LinearLayerConfig: two FP4 (E2M1) values per byte, one
+ *     FP8-E4M3 scale per 16 values, one global scale.
+ *
+ * Cache row (per token, per kv head, K or V): full_dim bytes =
+ *   [head_size/2 bytes: E2M1 pairs, element 2j in the low nibble of byte j]
+ *   [head_size/16 bytes: E4M3 block scales, one per 16 elements]
+ * Physical cache layout (HND): uint8 [num_blocks][2][num_kv_heads][block_size]
+ * [full_dim]; index 0 of the second dim is K, 1 is V. A page (block, K|V,
+ * head) is block_size*full_dim contiguous bytes.
+ *
+ * Quantization (bit-exact contract, g = k_scale or v_scale, fp32):
+ *   per group of 16: s32 = fl32(amax / fl32(6*g)); sb = E4M3 RNE satfinite(s32);
+ *   S = fl32(E4M3(sb) * g); code = E2M1 RNE satfinite(fl32(x / S)) (IEEE
+ *   division; sign kept, so small negatives give 0x8); S == 0 -> all codes 0.
+ * Dequantization: xhat = E2M1(code) * E4M3(sb) * g.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are caller-owned DEVICE memory unless stated; the library
+ *     never allocates device memory and never synchronizes the stream.
+ *   - Work is enqueued on `stream` (cudaStream_t; NULL = legacy default).
+ *   - Host-side validation failures return a negative status and launch
+ *     nothing. A CUDA launch error returns NVFP4_ERR_CUDA. Device-side faults
+ *     that the kernels detect (out-of-range block ids, a pipeline wait that
+ *     timed out) skip the bad access and raise bits in a device status word.
+ *   - bf16 tensors are passed as `const void*` (IEEE bfloat16 bit patterns).
+ *   - Supported: head_size in {64, 128, 256}; block_size in {16, 32};
+ *     num_q_heads / num_kv_heads in 1..8 (attention).
+ */
+#ifndef NVFP4KV_H_
+#define NVFP4KV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NVFP4KV_API __attribute__((visibility("default")))
+#else
+#define NVFP4KV_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad shape */
+  NVFP4_ERR_UNSUPPORTED = -2, /* valid but not built: head_size, block_size, GQA group */
+  NVFP4_ERR_CUDA = -3,        /* kernel launch / CUDA runtime error */
+  NVFP4_ERR_WORKSPACE = -4    /* workspace null or smaller than required */
+} nvfp4_status;
+
+/* Bits of the device status word (see nvfp4_paged_attention's workspace and
+ * nvfp4_quantize_append_paged's `device_status`). */
+#define NVFP4_DEV_BAD_SLOT 0x1u    /* slot >= num_blocks*block_size (token skipped) */
+#define NVFP4_DEV_BAD_BLOCK 0x2u   /* block id outside [0, num_blocks) (page skipped) */
+#define NVFP4_DEV_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
+
+/* Row width in bytes, head_size/2 + head_size/16 ("FlashInfer backend adds
+ * end-to-end NVFP4 KV cache support", get_kv_cache_shape, the
+ * nvfp4_kv_cache_full_dim helper). Returns -1 if head_size <= 0 or
+ * head_size % 16 != 0. Pure host function. */
+NVFP4KV_API int64_t nvfp4_kv_full_dim(int64_t head_size);
+
+/* Slot-mapped quantize-append ("FlashInfer backend adds end-to-end NVFP4 KV
+ * cache support", reshape_and_cache_flash with kv_cache_dtype "nvfp4";
+ * "FlashInfer NVFP4 KV serving on pre-SM100 GPUs", the slot-mapping append
+ * helper).
+ *   k, v            bf16 [num_tokens][num_kv_heads][head_size]; heads and
+ *                   elements contiguous, token stride given in ELEMENTS
+ *                   (>= num_kv_heads*head_size; allows views into a fused
+ *                   qkv buffer). 16-byte aligned rows required.
+ *   cache           uint8 HND cache, num_blocks*2*num_kv_heads*block_size*
+ *                   full_dim bytes, 16-byte aligned.
+ *   slot_mapping    int64 [num_tokens]; token t goes to block slot/block_size,
+ *                   offset slot%block_size; slot < 0 skips the token; a slot
+ *                   >= num_blocks*block_size is skipped and flagged.
+ *   k_scale,v_scale device fp32 scalars (global scales g; finite, > 0).
+ *   device_status   optional (NULL allowed) device uint32 word; the kernel
+ *                   ORs NVFP4_DEV_BAD_SLOT into it. Never cleared here.
+ * Rows not named by a slot are never touched. Duplicate slots: undefined
+ * which token wins. num_tokens == 0 is a no-op returning NVFP4_OK. */
+NVFP4KV_API int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_stride,
+                                int64_t v_token_stride, int64_t num_tokens,
+                                int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
+                                int64_t num_blocks, int32_t block_size,
+                                const int64_t* slot_mapping, const float* k_scale,
+                                const float* v_scale, uint32_t* device_status,
+                                nvfp4_stream_t stream);
+
+/* Bytes of workspace nvfp4_paged_attention needs for these sizes (a pure host
+ * function of its arguments). Returns 0 for invalid arguments. */
+NVFP4KV_API size_t nvfp4_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                            int32_t num_kv_heads, int32_t head_size);
+
+/* Paged decode and chunked-prefill attention over the NVFP4 cache ("FlashInfer
+ * backend adds end-to-end NVFP4 KV cache support", implementation breakdown
+ * items 2-3: FP8 output, dequantized back to the model dtype; the pages read
+ * through a block table with the split-out FP8 block scales).
+ *   q               bf16 [num_q_tokens][num_q_heads][head_size], token stride
+ *                   q_token_stride in elements, 16-byte aligned rows.
+ *   cache           HND cache as above.
+ *   block_table     int32 [num_seqs][max_blocks_per_seq]: logical block i of
+ *                   sequence b lives in cache block block_table[b][i].
+ *   seq_lens        int32 [num_seqs]: keys of sequence b (cached + new), >= 1.
+ *   qo_indptr       int32 [num_seqs+1] query-token ranges (chunked prefill and
+ *                   mixed batches), or NULL: one query token per sequence
+ *                   (token b of q belongs to sequence b; decode).
+ *                   Query row r of a sequence with q_len = qo_indptr[b+1] -
+ *                   qo_indptr[b] sits at position seq_lens[b]-q_len+r and sees
+ *                   keys 0..seq_lens[b]-q_len+r (causal); an empty window
+ *                   writes zeros.
+ *   max_q_len       host upper bound on every q_len (1 for pure decode).
+ *   kv_scales       device fp32 [2] = {k_scale, v_scale}.
+ *   sm_scale        softmax scale; <= 0 selects 1/sqrt(head_size).
+ *   o_fp8           uint8 E4M3 [num_q_tokens][num_q_heads][head_size]:
+ *                   E4M3 RNE satfinite(o / o_scale).
+ *   o_scale         device fp32 scalar (> 0).
+ *   o_bf16          optional bf16 output, same shape: bf16(E4M3(o_fp8)*o_scale).
+ *   o_f32           optional fp32 output of o before the FP8 cast (testing).
+ *   workspace       device scratch of >= nvfp4_paged_attention_workspace_size
+ *                   bytes, 256-byte aligned, ZERO-FILLED before its first use;
+ *                   every call that completes leaves it ready for the next
+ *                   one. Its first 4 bytes are the device status word
+ *                   (NVFP4_DEV_* bits, sticky until the caller clears them).
+ *                   Calls that share a workspace must not overlap on the GPU.
+ * The GQA group G = num_q_heads/num_kv_heads maps q head hq to kv head hq/G. */
+NVFP4KV_API int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                          int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                          int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                          const int32_t* block_table, int32_t max_blocks_per_seq,
+                          const int32_t* seq_lens, const int32_t* qo_indptr,
+                          int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                          float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                          void* o_bf16, float* o_f32, void* workspace,
+                          size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* Dequantize listed cache blocks to bf16 ("FlashInfer NVFP4 KV serving on
+ * pre-SM100 GPUs", quick answer: the paged NVFP4 dequantize helper).
+ *   block_ids       int32 [num_block_ids]: cache blocks to expand.
+ *   kv_scales       device fp32 [2] = {k_scale, v_scale}.
+ *   out_bf16        bf16 [num_block_ids][2][num_kv_heads][block_size][head_size]:
+ *                   out[i] = bf16_RNE(fl32(xhat * g)) of block block_ids[i].
+ * Out-of-range block ids are skipped (output left untouched). */
+NVFP4KV_API int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks, int32_t block_size,
+                           int32_t num_kv_heads, int32_t head_size,
+                           const int32_t* block_ids, int64_t num_block_ids,
+                           const float* kv_scales, void* out_bf16, nvfp4_stream_t stream);
+
+/* Static description of a status code. */
+NVFP4KV_API const char* nvfp4_status_string(int status);
+
+/* Text of the CUDA error behind the calling thread's most recent
+ * NVFP4_ERR_CUDA ("no error" if none). Static string, not owned by caller. */
+NVFP4KV_API const char* nvfp4_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4KV_H_ */

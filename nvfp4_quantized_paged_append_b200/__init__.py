@@ -1,0 +1,197 @@
+"""NVFP4 paged KV cache for B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/nvfp4kv.h`` (``libnvfp4kv.so``,
+built in-tree by ``python -m nvfp4_quantized_paged_append_b200.build``).
+Every function below only marshals torch tensors into pointers, sizes and the
+current CUDA stream; all work runs in the library's kernels. There is no CPU
+fallback: if the library is missing, the first call into it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4kv.so")
+
+NVFP4_OK = 0
+NVFP4_ERR_INVALID_ARG = -1
+NVFP4_ERR_UNSUPPORTED = -2
+NVFP4_ERR_CUDA = -3
+NVFP4_ERR_WORKSPACE = -4
+
+DEV_BAD_SLOT = 0x1
+DEV_BAD_BLOCK = 0x2
+DEV_TIMEOUT = 0x4
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        msg = f"{what}: {status_string(status)} ({status})"
+        if status == NVFP4_ERR_CUDA:
+            msg += f": {lib().nvfp4_last_cuda_error().decode()}"
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvfp4kv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m nvfp4_quantized_paged_append_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, f32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
+                            ctypes.c_size_t)
+    L.nvfp4_kv_full_dim.argtypes = [i64]
+    L.nvfp4_kv_full_dim.restype = i64
+    L.nvfp4_status_string.argtypes = [ctypes.c_int]
+    L.nvfp4_status_string.restype = ctypes.c_char_p
+    L.nvfp4_last_cuda_error.argtypes = []
+    L.nvfp4_last_cuda_error.restype = ctypes.c_char_p
+    L.nvfp4_quantize_append_paged.argtypes = [P, P, i64, i64, i64, i32, i32, P, i64, i32, P, P, P,
+                                              P, P]
+    L.nvfp4_quantize_append_paged.restype = ctypes.c_int
+    L.nvfp4_paged_attention_workspace_size.argtypes = [i32, i32, i32, i32]
+    L.nvfp4_paged_attention_workspace_size.restype = sz
+    L.nvfp4_paged_attention.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P, i32, P, P,
+                                        i32, i32, P, f32, P, P, P, P, P, sz, P]
+    L.nvfp4_paged_attention.restype = ctypes.c_int
+    L.nvfp4_dequantize_paged.argtypes = [P, i64, i32, i32, i32, P, i64, P, P, P]
+    L.nvfp4_dequantize_paged.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4_status_string(status).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != NVFP4_OK:
+        raise Nvfp4Error(status, what)
+
+
+def full_dim(head_size: int) -> int:
+    """head_size/2 + head_size/16 bytes per cache row (-1 if invalid)."""
+    return int(lib().nvfp4_kv_full_dim(head_size))
+
+
+def kv_cache_shape(num_blocks: int, block_size: int, num_kv_heads: int, head_size: int):
+    """Logical (NHD) shape of the cache: (num_blocks, 2, block_size, num_kv_heads, full_dim)."""
+    return (num_blocks, 2, block_size, num_kv_heads, full_dim(head_size))
+
+
+def alloc_kv_cache(num_blocks: int, block_size: int, num_kv_heads: int, head_size: int,
+                   device="cuda") -> torch.Tensor:
+    """uint8 cache in HND storage order: (num_blocks, 2, num_kv_heads, block_size, full_dim)."""
+    return torch.zeros((num_blocks, 2, num_kv_heads, block_size, full_dim(head_size)),
+                       dtype=torch.uint8, device=device)
+
+
+def _cache_dims(cache: torch.Tensor):
+    if cache.dtype != torch.uint8 or cache.dim() != 5 or cache.shape[1] != 2 or not cache.is_contiguous():
+        raise ValueError("cache must be a contiguous uint8 HND tensor (NB, 2, Hkv, bs, full_dim)")
+    nb, _, hkv, bs, f = cache.shape
+    d = f * 16 // 9
+    if full_dim(d) != f:
+        raise ValueError(f"cache last dim {f} is not a valid full_dim")
+    return nb, hkv, bs, d
+
+
+def quantize_append_paged(k: torch.Tensor, v: torch.Tensor, cache: torch.Tensor,
+                          slot_mapping: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                          device_status: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Quantize bf16 k/v [T, Hkv, D] into the NVFP4 HND cache at slot_mapping."""
+    nb, hkv, bs, d = _cache_dims(cache)
+    T = slot_mapping.shape[0]
+    for name, x in (("k", k), ("v", v)):
+        if x.dtype != torch.bfloat16 or x.shape != (T, hkv, d) or x.stride(2) != 1 or x.stride(1) != d:
+            raise ValueError(f"{name} must be bf16 [T, {hkv}, {d}] with contiguous heads")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    st = lib().nvfp4_quantize_append_paged(
+        _ptr(k), _ptr(v), k.stride(0), v.stride(0), T, hkv, d, _ptr(cache), nb, bs,
+        _ptr(slot_mapping), _ptr(k_scale), _ptr(v_scale), _ptr(device_status), _stream(stream))
+    _check(st, "nvfp4_quantize_append_paged")
+
+
+def workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_size: int) -> int:
+    return int(lib().nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                          head_size))
+
+
+def alloc_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_size: int,
+                    device="cuda") -> torch.Tensor:
+    """Zero-filled workspace (uint8). Its first 4 bytes are the device status word."""
+    n = workspace_size(num_seqs, num_q_heads, num_kv_heads, head_size)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_status(workspace: torch.Tensor) -> int:
+    """Device status bits (DEV_*) recorded in a workspace (synchronizes)."""
+    return int(workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
+
+
+def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
+                    seq_lens: torch.Tensor, kv_scales: torch.Tensor, o_fp8: torch.Tensor,
+                    o_scale: torch.Tensor, workspace: torch.Tensor,
+                    qo_indptr: Optional[torch.Tensor] = None, max_q_len: int = 1,
+                    sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
+                    o_f32: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32)."""
+    nb, hkv, bs, d = _cache_dims(cache)
+    tq, hq, dq = q.shape
+    if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
+        raise ValueError("q must be bf16 [Tq, Hq, D] with contiguous heads")
+    B, mb = block_table.shape
+    if block_table.dtype != torch.int32 or not block_table.is_contiguous():
+        raise ValueError("block_table must be contiguous int32 [B, max_blocks]")
+    if seq_lens.dtype != torch.int32 or qo_indptr is not None and qo_indptr.dtype != torch.int32:
+        raise ValueError("seq_lens / qo_indptr must be int32")
+    for name, o, dt in (("o_fp8", o_fp8, torch.uint8), ("o_bf16", o_bf16, torch.bfloat16),
+                        ("o_f32", o_f32, torch.float32)):
+        if o is not None and (o.dtype != dt or o.shape != (tq, hq, d) or not o.is_contiguous()):
+            raise ValueError(f"{name} must be contiguous {dt} [Tq, Hq, D]")
+    st = lib().nvfp4_paged_attention(
+        _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
+        _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
+        _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "nvfp4_paged_attention")
+
+
+def dequantize_paged(cache: torch.Tensor, block_ids: torch.Tensor, kv_scales: torch.Tensor,
+                     out: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """bf16 [len(block_ids), 2, Hkv, bs, D] pages of the listed blocks."""
+    nb, hkv, bs, d = _cache_dims(cache)
+    n = block_ids.shape[0]
+    if out is None:
+        out = torch.empty((n, 2, hkv, bs, d), dtype=torch.bfloat16, device=cache.device)
+    if block_ids.dtype != torch.int32:
+        raise ValueError("block_ids must be int32")
+    st = lib().nvfp4_dequantize_paged(_ptr(cache), nb, bs, hkv, d, _ptr(block_ids), n,
+                                      _ptr(kv_scales), _ptr(out), _stream(stream))
+    _check(st, "nvfp4_dequantize_paged")
+    return out

@@ -1,0 +1,170 @@
+// C ABI of libnvfp4kv: host-side validation, then kernel launches on the
+// caller's stream. See include/nvfp4kv.h for the contract of each call.
+#include <math.h>
+
+#include "../../include/nvfp4kv.h"
+#include "nvfp4kv_launch.h"
+
+namespace nvfp4kv {
+size_t decode_smem_bytes(int head_size, int block_size, int num_seqs);
+}
+
+namespace {
+
+bool head_size_ok(int64_t d) { return d == 64 || d == 128 || d == 256; }
+bool block_size_ok(int64_t bs) { return bs == 16 || bs == 32; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+thread_local const char* g_last_error = "no error";
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return NVFP4_OK;
+  g_last_error = cudaGetErrorString(e);
+  return NVFP4_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t nvfp4_kv_full_dim(int64_t head_size) {
+  if (head_size <= 0 || head_size % 16 != 0) return -1;
+  return head_size / 2 + head_size / 16;
+}
+
+const char* nvfp4_last_cuda_error(void) { return g_last_error; }
+
+const char* nvfp4_status_string(int status) {
+  switch (status) {
+    case NVFP4_OK:
+      return "ok";
+    case NVFP4_ERR_INVALID_ARG:
+      return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED:
+      return "unsupported configuration";
+    case NVFP4_ERR_CUDA:
+      return "CUDA error";
+    case NVFP4_ERR_WORKSPACE:
+      return "workspace missing or too small";
+    default:
+      return "unknown status";
+  }
+}
+
+int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_stride,
+                                int64_t v_token_stride, int64_t num_tokens,
+                                int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
+                                int64_t num_blocks, int32_t block_size,
+                                const int64_t* slot_mapping, const float* k_scale,
+                                const float* v_scale, uint32_t* device_status,
+                                nvfp4_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_size <= 0 || num_blocks <= 0 ||
+      block_size <= 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (head_size % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!head_size_ok(head_size) || !block_size_ok(block_size)) return NVFP4_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return NVFP4_OK;
+  if (!k || !v || !cache || !slot_mapping || !k_scale || !v_scale) return NVFP4_ERR_INVALID_ARG;
+  const int64_t row = (int64_t)num_kv_heads * head_size;
+  if (k_token_stride < row || v_token_stride < row || k_token_stride % 8 != 0 ||
+      v_token_stride % 8 != 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(cache, 16) || !aligned(slot_mapping, 8))
+    return NVFP4_ERR_INVALID_ARG;
+  nvfp4kv::QuantizeAppendArgs a{k,           v,          k_token_stride, v_token_stride,
+                                num_tokens,  num_kv_heads, head_size,    cache,
+                                num_blocks,  block_size, slot_mapping,   k_scale,
+                                v_scale,     device_status};
+  return cuda_status(nvfp4kv::launch_quantize_append(a, (cudaStream_t)stream));
+}
+
+size_t nvfp4_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                            int32_t num_kv_heads, int32_t head_size) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_size <= 0) return 0;
+  return nvfp4kv::workspace_layout(num_seqs, num_kv_heads, head_size).total;
+}
+
+int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                          int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                          int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                          const int32_t* block_table, int32_t max_blocks_per_seq,
+                          const int32_t* seq_lens, const int32_t* qo_indptr,
+                          int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                          float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                          void* o_bf16, float* o_f32, void* workspace,
+                          size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (num_q_tokens < 0 || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
+      max_q_len < 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (head_size % 16 != 0 || num_q_heads % num_kv_heads != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!head_size_ok(head_size) || !block_size_ok(block_size)) return NVFP4_ERR_UNSUPPORTED;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > 8) return NVFP4_ERR_UNSUPPORTED;
+  if (!qo_indptr && num_q_tokens < num_seqs) return NVFP4_ERR_INVALID_ARG;
+  if (!qo_indptr && max_q_len > 1) return NVFP4_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_q_tokens == 0) return NVFP4_OK;
+  if (!q || !cache || !block_table || !seq_lens || !kv_scales || !o_fp8 || !o_scale)
+    return NVFP4_ERR_INVALID_ARG;
+  if (q_token_stride < (int64_t)num_q_heads * head_size || q_token_stride % 8 != 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(cache, 16) || (o_bf16 && !aligned(o_bf16, 2)) ||
+      (o_f32 && !aligned(o_f32, 4)))
+    return NVFP4_ERR_INVALID_ARG;
+  // flattened page indices are int32 on the device
+  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
+    return NVFP4_ERR_UNSUPPORTED;
+  if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs) > 226 * 1024)
+    return NVFP4_ERR_UNSUPPORTED;
+  const size_t need = nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                           head_size);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return NVFP4_ERR_WORKSPACE;
+
+  nvfp4kv::AttentionArgs a{};
+  a.q = q;
+  a.q_token_stride = q_token_stride;
+  a.num_q_tokens = num_q_tokens;
+  a.num_q_heads = num_q_heads;
+  a.cache = cache;
+  a.num_blocks = num_blocks;
+  a.block_size = block_size;
+  a.num_kv_heads = num_kv_heads;
+  a.head_size = head_size;
+  a.block_table = block_table;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.seq_lens = seq_lens;
+  a.qo_indptr = qo_indptr;
+  a.num_seqs = num_seqs;
+  a.max_q_len = max_q_len;
+  a.kv_scales = kv_scales;
+  a.sm_scale = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)head_size);
+  a.o_fp8 = o_fp8;
+  a.o_scale = o_scale;
+  a.o_bf16 = o_bf16;
+  a.o_f32 = o_f32;
+  a.workspace = workspace;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int st = cuda_status(nvfp4kv::launch_decode_attention(a, s));
+  if (st != NVFP4_OK) return st;
+  if (qo_indptr && max_q_len > 1) return cuda_status(nvfp4kv::launch_prefill_attention(a, s));
+  return NVFP4_OK;
+}
+
+int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks, int32_t block_size,
+                           int32_t num_kv_heads, int32_t head_size,
+                           const int32_t* block_ids, int64_t num_block_ids,
+                           const float* kv_scales, void* out_bf16, nvfp4_stream_t stream) {
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_size <= 0 ||
+      num_block_ids < 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (head_size % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!head_size_ok(head_size) || !block_size_ok(block_size)) return NVFP4_ERR_UNSUPPORTED;
+  if (num_block_ids == 0) return NVFP4_OK;
+  if (!cache || !block_ids || !kv_scales || !out_bf16) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(cache, 16) || !aligned(out_bf16, 16)) return NVFP4_ERR_INVALID_ARG;
+  nvfp4kv::DequantArgs a{cache, num_blocks, block_size, num_kv_heads, head_size,
+                         block_ids, num_block_ids, kv_scales, out_bf16};
+  return cuda_status(nvfp4kv::launch_dequantize_paged(a, (cudaStream_t)stream));
+}
+
+}  // extern "C"

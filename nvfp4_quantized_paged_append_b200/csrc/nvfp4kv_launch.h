@@ -1,0 +1,85 @@
+// Host-side launch interface between the C ABI (api.cu) and the kernels.
+// Arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nvfp4kv {
+
+struct QuantizeAppendArgs {
+  const void* k;
+  const void* v;
+  int64_t k_token_stride, v_token_stride, num_tokens;
+  int num_kv_heads, head_size;
+  uint8_t* cache;
+  int64_t num_blocks;
+  int block_size;
+  const int64_t* slot_mapping;
+  const float* k_scale;
+  const float* v_scale;
+  uint32_t* device_status;
+};
+
+struct DequantArgs {
+  const uint8_t* cache;
+  int64_t num_blocks;
+  int block_size, num_kv_heads, head_size;
+  const int32_t* block_ids;
+  int64_t num_block_ids;
+  const float* kv_scales;
+  void* out_bf16;
+};
+
+struct AttentionArgs {
+  const void* q;
+  int64_t q_token_stride, num_q_tokens;
+  int num_q_heads;
+  const uint8_t* cache;
+  int64_t num_blocks;
+  int block_size, num_kv_heads, head_size;
+  const int32_t* block_table;
+  int max_blocks_per_seq;
+  const int32_t* seq_lens;
+  const int32_t* qo_indptr;  // may be null (decode)
+  int num_seqs, max_q_len;
+  const float* kv_scales;
+  float sm_scale;  // resolved (> 0)
+  uint8_t* o_fp8;
+  const float* o_scale;
+  void* o_bf16;   // may be null
+  float* o_f32;   // may be null
+  void* workspace;
+};
+
+// Decode split-KV grid: CTAs launched for the flattened page range. The
+// workspace holds two partial-state slots per CTA.
+constexpr int kDecodeCtas = 148 * 4;
+
+// Workspace layout (bytes from the start, all 256-byte aligned):
+//   [0, 256)                     uint32 device status word (+ padding)
+//   counters: int32 [num_seqs * num_kv_heads]
+//   partials: float [kDecodeCtas * 2][8 rows][head_size] accumulators
+//   partial m/l: float [kDecodeCtas * 2][8 rows][2]
+struct WorkspaceLayout {
+  size_t counters_off, partials_off, ml_off, total;
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads, int head_size) {
+  WorkspaceLayout w;
+  w.counters_off = 256;
+  w.partials_off = align256(w.counters_off + sizeof(int32_t) * (size_t)num_seqs * num_kv_heads);
+  w.ml_off = align256(w.partials_off + sizeof(float) * (size_t)kDecodeCtas * 2 * 8 * head_size);
+  w.total = align256(w.ml_off + sizeof(float) * (size_t)kDecodeCtas * 2 * 8 * 2);
+  return w;
+}
+
+cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t stream);
+cudaError_t launch_dequantize_paged(const DequantArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_attention(const AttentionArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_attention(const AttentionArgs& a, cudaStream_t stream);
+
+}  // namespace nvfp4kv

@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point the header declares, and rejects bad arguments before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_quantized_paged_append_b200 as nk
+from nvfp4_quantized_paged_append_b200 import build as nkbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nkbuild.build()
+    return nk.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "nvfp4kv.h")).read()
+    return re.findall(r"NVFP4KV_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert len(names) >= 6
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_full_dim(L):
+    assert [nk.full_dim(d) for d in (16, 64, 128, 256)] == [9, 36, 72, 144]
+    assert nk.full_dim(0) == -1 and nk.full_dim(100) == -1 and nk.full_dim(-16) == -1
+
+
+def test_status_strings(L):
+    for s in (0, -1, -2, -3, -4):
+        assert nk.status_string(s)
+    assert nk.status_string(-99) == "unknown status"
+
+
+def _append(L, **kw):
+    a = dict(k=None, v=None, ks=128 * 8, vs=128 * 8, T=4, H=8, D=128, cache=None, nb=10, bs=16,
+             slots=None, kscale=None, vscale=None, status=None, stream=None)
+    a.update(kw)
+    P = ctypes.c_void_p
+    return L.nvfp4_quantize_append_paged(a["k"], a["v"], a["ks"], a["vs"], a["T"], a["H"], a["D"],
+                                         a["cache"], a["nb"], a["bs"], a["slots"], a["kscale"],
+                                         a["vscale"], a["status"], a["stream"])
+
+
+def test_append_validation(L):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    assert _append(L) == nk.NVFP4_ERR_INVALID_ARG                      # null pointers
+    assert _append(L, T=0) == nk.NVFP4_OK                              # empty: no-op
+    assert _append(L, D=100) == nk.NVFP4_ERR_INVALID_ARG
+    assert _append(L, D=96) == nk.NVFP4_ERR_UNSUPPORTED
+    assert _append(L, bs=8) == nk.NVFP4_ERR_UNSUPPORTED
+    assert _append(L, T=-1) == nk.NVFP4_ERR_INVALID_ARG
+    full = dict(k=fake, v=fake, cache=fake, slots=fake, kscale=fake, vscale=fake)
+    assert _append(L, ks=100, **full) == nk.NVFP4_ERR_INVALID_ARG      # stride < row
+    assert _append(L, ks=1028, **full) == nk.NVFP4_ERR_INVALID_ARG     # stride not 16-B multiple
+    assert _append(L, **dict(full, k=ctypes.c_void_p(0x1002))) == nk.NVFP4_ERR_INVALID_ARG  # misaligned
+
+
+def _attn(L, **kw):
+    a = dict(q=None, qs=16 * 128, tq=4, hq=16, cache=None, nb=10, bs=16, hkv=8, D=128, bt=None,
+             mb=4, sl=None, qo=None, B=4, mq=1, kvs=None, sm=0.0, o8=None, osc=None, o16=None,
+             o32=None, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return L.nvfp4_paged_attention(a["q"], a["qs"], a["tq"], a["hq"], a["cache"], a["nb"], a["bs"],
+                                   a["hkv"], a["D"], a["bt"], a["mb"], a["sl"], a["qo"], a["B"],
+                                   a["mq"], a["kvs"], a["sm"], a["o8"], a["osc"], a["o16"],
+                                   a["o32"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_attention_validation(L):
+    fake = ctypes.c_void_p(0x1000)
+    full = dict(q=fake, cache=fake, bt=fake, sl=fake, kvs=fake, o8=fake, osc=fake)
+    assert _attn(L) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn(L, B=0) == nk.NVFP4_OK
+    assert _attn(L, hq=12) == nk.NVFP4_ERR_INVALID_ARG          # Hq % Hkv
+    assert _attn(L, hq=128) == nk.NVFP4_ERR_UNSUPPORTED         # G = 16
+    assert _attn(L, D=96, qs=16 * 96) == nk.NVFP4_ERR_UNSUPPORTED
+    assert _attn(L, mq=4) == nk.NVFP4_ERR_INVALID_ARG           # prefill needs qo_indptr
+    assert _attn(L, tq=2) == nk.NVFP4_ERR_INVALID_ARG           # decode needs one q per seq
+    assert _attn(L, **full) == nk.NVFP4_ERR_WORKSPACE           # no workspace
+    need = nk.workspace_size(4, 16, 8, 128)
+    assert need > 0 and need % 256 == 0
+    assert _attn(L, ws=ctypes.c_void_p(0x100000), wsb=need - 1, **full) == nk.NVFP4_ERR_WORKSPACE
+    assert _attn(L, ws=ctypes.c_void_p(0x100010), wsb=need, **full) == nk.NVFP4_ERR_WORKSPACE  # alignment
+
+
+def test_workspace_size_monotone(L):
+    assert nk.workspace_size(1, 16, 8, 128) <= nk.workspace_size(64, 16, 8, 128)
+    assert nk.workspace_size(8, 64, 8, 256) > nk.workspace_size(8, 64, 8, 128)
+    assert nk.workspace_size(-1, 16, 8, 128) == 0
+
+
+def test_dequant_validation(L):
+    P = ctypes.c_void_p
+    f = L.nvfp4_dequantize_paged
+    assert f(None, 10, 16, 8, 128, None, 4, None, None, None) == nk.NVFP4_ERR_INVALID_ARG
+    assert f(None, 10, 16, 8, 128, None, 0, None, None, None) == nk.NVFP4_OK
+    assert f(None, 10, 16, 8, 48, None, 4, None, None, None) == nk.NVFP4_ERR_UNSUPPORTED

@@ -1,0 +1,149 @@
+"""Paged attention on the GPU vs the fp64 CPU oracle.
+
+Bar: per output row (query token, head) max |o - o_ref| <= 2e-3 * max |o_ref|
+before the FP8 cast (o_f32), E4M3 output within one step of the oracle's
+E4M3(o_ref / o_scale), and o_bf16 equal to bf16(E4M3 * o_scale) of such a code.
+Every workload runs at full size on the GPU in the launch configuration the
+benchmark uses; the oracle checks all rows of the smaller ones and sampled
+sequences / query rows of the two largest."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_quantized_paged_append_b200 as nk
+from nvfp4_quantized_paged_append_b200 import workloads as wl
+from paged_helpers import (build_gpu_cache, check_bf16_from_fp8, check_fp8, check_rows, oracle_case,
+                           run_gpu_attention, run_oracle)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _compare(w, scales, gpu_out, case, ref):
+    o8, o16, o32 = (t.cpu() for t in gpu_out)
+    idx = case["out_index"]
+    o64, r8, _ = ref
+    hq, d = w.num_q_heads, w.head_size
+    g32 = o32.numpy()[idx].reshape(-1, d)
+    worst = check_rows(g32, o64.reshape(-1, d))
+    check_fp8(o8.numpy()[idx], r8)
+    check_bf16_from_fp8(o16.contiguous().view(torch.int16).numpy().view(np.uint16)[idx], r8, scales[2])
+    assert np.isfinite(g32).all()
+    return worst
+
+
+@pytest.mark.parametrize("name", ["tiny_decode", "qwen3_0p6b_decode"])
+def test_decode_workload_full(name):
+    w = wl.make_workload(name)
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.workspace_status(out[3]) == 0
+    case = oracle_case(w, range(w.num_seqs), scales, DEV)
+    _compare(w, scales, out[:3], case, run_oracle(case, scales))
+
+
+def test_long_decode_sampled():
+    w = wl.make_workload("long_decode")
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.workspace_status(out[3]) == 0
+    case = oracle_case(w, [0, 31, 63], scales, DEV)
+    _compare(w, scales, out[:3], case, run_oracle(case, scales))
+
+
+def test_mixed_prefill_decode_sampled():
+    w = wl.make_workload("mixed_prefill_decode")
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.workspace_status(out[3]) == 0
+    rows = {0: [0, 1, 7, 8, 63, 64, 1023, 2047], 7: [2, 500, 1500, 2046]}
+    case = oracle_case(w, [0, 7, 8, 30, 63], scales, DEV, rows=rows)
+    _compare(w, scales, out[:3], case, run_oracle(case, scales))
+
+
+EDGE = [
+    # (D, bs, Hq, Hkv, seq_lens, q_lens)
+    (128, 16, 16, 8, [1, 16, 17, 33, 500], None),          # page edges, single key
+    (64, 32, 8, 8, [1, 31, 32, 65], None),                  # G = 1, bs 32
+    (256, 16, 64, 8, [3, 129, 1000], None),                 # G = 8, D 256
+    (128, 32, 32, 8, [4096, 7], None),                      # G = 4
+    (64, 16, 4, 2, [37, 100], [5, 1]),                       # prefill + decode mix
+    (128, 16, 16, 8, [40, 300, 16], [40, 77, 2]),           # q_len == L (no cache) / ragged
+    (256, 32, 16, 2, [200, 64], [130, 64]),                 # G = 8, bs 32 prefill
+    (128, 16, 8, 2, [5], [9]),                              # q_len > L: early rows see nothing
+]
+
+
+@pytest.mark.parametrize("D,bs,hq,hkv,lens,qlens", EDGE)
+def test_edge_cases(D, bs, hq, hkv, lens, qlens):
+    w = wl.custom_workload("edge", 100 + D + bs + len(lens), hq, hkv, D, bs, lens, qlens,
+                           outliers="x20", spare_blocks=3)
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.workspace_status(out[3]) == 0
+    case = oracle_case(w, range(w.num_seqs), scales, DEV)
+    _compare(w, scales, out[:3], case, run_oracle(case, scales))
+
+
+def test_repeat_calls_identical_and_workspace_reusable():
+    """Split-KV tickets reset themselves: a second call on the same workspace
+    gives bit-identical outputs."""
+    w = wl.make_workload("qwen3_0p6b_decode")
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    q = wl.queries(w, DEV)
+    k_scale, v_scale, o_scale = scales
+    ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, DEV)
+    bt = torch.from_numpy(w.block_table).to(DEV)
+    sl = torch.from_numpy(w.seq_lens).to(DEV)
+    kvs = torch.tensor([k_scale, v_scale], dtype=torch.float32, device=DEV)
+    osc = torch.tensor([o_scale], dtype=torch.float32, device=DEV)
+    outs = []
+    for _ in range(3):
+        o8 = torch.empty((w.num_seqs, w.num_q_heads, w.head_size), dtype=torch.uint8, device=DEV)
+        o32 = torch.empty((w.num_seqs, w.num_q_heads, w.head_size), dtype=torch.float32, device=DEV)
+        nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, o_f32=o32)
+        outs.append((o8.clone(), o32.clone()))
+    torch.cuda.synchronize()
+    for o8, o32 in outs[1:]:
+        assert torch.equal(o8, outs[0][0]) and torch.equal(o32, outs[0][1])
+    # counters are back to zero
+    lay_counters = ws[256: 256 + 4 * w.num_seqs * w.num_kv_heads].view(torch.int32)
+    assert int(lay_counters.abs().sum()) == 0
+
+
+def test_bad_block_id_flagged_no_fault():
+    w = wl.custom_workload("badblk", 5, 8, 2, 128, 16, [40, 70])
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    w.block_table[1, 2] = w.num_blocks + 1000   # out of range
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.workspace_status(out[3]) & nk.DEV_BAD_BLOCK
+    assert torch.isfinite(out[2]).all()
+
+
+def test_output_scale_and_sm_scale_arguments():
+    """A non-default sm_scale and a small o_scale (saturating FP8) behave as specified."""
+    w = wl.make_workload("tiny_decode")
+    scales = (1.0, 1.0, 0.002)
+    cache = build_gpu_cache(w, scales, DEV)
+    q = wl.queries(w, DEV)
+    o8 = torch.empty((2, 4, 64), dtype=torch.uint8, device=DEV)
+    o32 = torch.empty((2, 4, 64), dtype=torch.float32, device=DEV)
+    ws = nk.alloc_workspace(2, 4, 2, 64, DEV)
+    nk.paged_attention(q, cache, torch.from_numpy(w.block_table).to(DEV),
+                       torch.from_numpy(w.seq_lens).to(DEV), torch.ones(2, device=DEV), o8,
+                       torch.tensor([0.002], device=DEV), ws, sm_scale=0.3, o_f32=o32)
+    torch.cuda.synchronize()
+    case = oracle_case(w, [0, 1], scales, DEV)
+    import oracle
+    o64, r8, _ = oracle.paged_attention(case["q"], case["cache"], case["block_table"],
+                                        case["seq_lens"], None, 1.0, 1.0, 0.3, 0.002)
+    check_rows(o32.cpu().numpy().reshape(-1, 64), o64.reshape(-1, 64))
+    check_fp8(o8.cpu().numpy(), r8)
+    assert ((r8.astype(np.int64) & 0x7F) == 0x7E).any()        # some outputs saturate at 448
+    assert ((o8.cpu().numpy().astype(np.int64) & 0x7F) == 0x7E).any()
