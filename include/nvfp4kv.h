@@ -167,6 +167,34 @@ NVFP4KV_API int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
                            const int32_t* block_ids, int64_t num_block_ids,
                            const float* kv_scales, void* out_bf16, nvfp4_stream_t stream);
 
+/* Paged attention that allocates nothing and takes no workspace. The pages
+ * this library follows have no counterpart: it exists for callers that
+ * cannot provide the scratch memory nvfp4_paged_attention asks for, such as
+ * code handed only its input and output buffers by a host framework (a
+ * plugin or callback interface with no workspace hook), or code running
+ * while all device memory is owned by an allocator it may not draw from.
+ * Arguments and results are those of nvfp4_paged_attention without
+ * `workspace` / `workspace_bytes`; the caller still provides every input and
+ * output buffer.
+ * Scratch: one fixed array of NVFP4_NOALLOC_SCRATCH_BYTES bytes in device
+ * memory, defined inside the library; every GPU that loads the library keeps
+ * it until the process exits. Sizes whose workspace
+ * (nvfp4_paged_attention_workspace_size) exceeds it return
+ * NVFP4_ERR_WORKSPACE. The first call on a device looks up the array's
+ * device address on that device (make that first call before any stream
+ * capture). Each call clears the array's status word and completion tickets
+ * on `stream` first; all calls share the one array, so calls that may
+ * overlap on the GPU (unordered streams) race and must not be made. The
+ * call never calls cudaMalloc, cudaFree or any allocating routine. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)12 << 20)
+NVFP4KV_API int nvfp4_paged_attention_noalloc(
+    const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
+    const uint8_t* cache, int64_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+    int32_t head_size, const int32_t* block_table, int32_t max_blocks_per_seq,
+    const int32_t* seq_lens, const int32_t* qo_indptr, int32_t num_seqs, int32_t max_q_len,
+    const float* kv_scales, float sm_scale, uint8_t* o_fp8, const float* o_scale,
+    void* o_bf16, float* o_f32, nvfp4_stream_t stream);
+
 /* Static description of a status code. */
 NVFP4KV_API const char* nvfp4_status_string(int status);
 

@@ -66,6 +66,9 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_paged_attention.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P, i32, P, P,
                                         i32, i32, P, f32, P, P, P, P, P, sz, P]
     L.nvfp4_paged_attention.restype = ctypes.c_int
+    L.nvfp4_paged_attention_noalloc.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P,
+                                                i32, P, P, i32, i32, P, f32, P, P, P, P, P]
+    L.nvfp4_paged_attention_noalloc.restype = ctypes.c_int
     L.nvfp4_dequantize_paged.argtypes = [P, i64, i32, i32, i32, P, i64, P, P, P]
     L.nvfp4_dequantize_paged.restype = ctypes.c_int
     _lib = L
@@ -179,6 +182,29 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
         _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "nvfp4_paged_attention")
+
+
+def paged_attention_noalloc(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
+                            seq_lens: torch.Tensor, kv_scales: torch.Tensor, o_fp8: torch.Tensor,
+                            o_scale: torch.Tensor, qo_indptr: Optional[torch.Tensor] = None,
+                            max_q_len: int = 1, sm_scale: float = 0.0,
+                            o_bf16: Optional[torch.Tensor] = None,
+                            o_f32: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None) -> None:
+    """paged_attention for callers that cannot hand over a workspace: the
+    library uses its own fixed scratch array (see nvfp4_paged_attention_noalloc
+    in include/nvfp4kv.h: one array per GPU, shared by all calls, so calls must
+    not overlap on the GPU; sizes beyond it raise)."""
+    nb, hkv, bs, d = _cache_dims(cache)
+    tq, hq, dq = q.shape
+    if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
+        raise ValueError("q must be bf16 [Tq, Hq, D] with contiguous heads")
+    B, mb = block_table.shape
+    st = lib().nvfp4_paged_attention_noalloc(
+        _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
+        _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
+        _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _stream(stream))
+    _check(st, "nvfp4_paged_attention_noalloc")
 
 
 def dequantize_paged(cache: torch.Tensor, block_ids: torch.Tensor, kv_scales: torch.Tensor,
