@@ -54,6 +54,10 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", choices=["attention", "append"], default=None,
+                   help="kernel-only mode for profilers: set up, then launch the chosen "
+                        "kernel --steps times (no timing, no JSON)")
+    p.add_argument("--workload", default=WORKLOAD, help="workload for --profile attention")
     return p.parse_args()
 
 
@@ -505,8 +509,54 @@ def run_reference(args, rank, world):
     }
 
 
+def run_profile(args):
+    """Set up one workload and launch one kernel --steps times (for ncu)."""
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    if args.profile == "append":
+        app = wl.make_append()
+        k, v = app.kv(dev)
+        gk, gv = app.scales(k, v)
+        slots = torch.from_numpy(app.slot_mapping()).to(dev)
+        cache = nk.alloc_kv_cache(app.num_blocks, app.block_size, app.num_kv_heads,
+                                  app.head_size, dev)
+        ks = torch.tensor([gk], device=dev)
+        vs = torch.tensor([gv], device=dev)
+        for _ in range(args.steps):
+            nk.quantize_append_paged(k, v, cache, slots, ks, vs)
+    else:
+        w = wl.make_workload(args.workload)
+        scales = wl.global_scales(w, dev)
+        cache = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+        ks = torch.tensor([scales[0]], device=dev)
+        vs = torch.tensor([scales[1]], device=dev)
+        for b in range(w.num_seqs):
+            k, v = wl.seq_kv(w, b, dev)
+            nk.quantize_append_paged(k, v, cache, torch.from_numpy(w.slots_for_seq(b)).to(dev),
+                                     ks, vs)
+        q = wl.queries(w, dev)
+        o8 = torch.empty((w.num_q_tokens, w.num_q_heads, w.head_size), dtype=torch.uint8,
+                         device=dev)
+        ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, dev)
+        bt = torch.from_numpy(w.block_table).to(dev)
+        sl = torch.from_numpy(w.seq_lens).to(dev)
+        qo = None if w.is_decode else torch.from_numpy(w.qo_indptr).to(dev)
+        kvs = torch.tensor([scales[0], scales[1]], device=dev)
+        osc = torch.tensor([scales[2]], device=dev)
+        for _ in range(args.steps):
+            nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, qo_indptr=qo,
+                               max_q_len=w.max_q_len)
+    torch.cuda.synchronize()
+    print(f"profile mode: {args.profile} x{args.steps} done", flush=True)
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))

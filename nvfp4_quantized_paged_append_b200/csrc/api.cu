@@ -81,7 +81,9 @@ int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_st
 size_t nvfp4_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                             int32_t num_kv_heads, int32_t head_size) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_size <= 0) return 0;
-  return nvfp4kv::workspace_layout(num_seqs, num_kv_heads, head_size).total;
+  if (num_q_heads % num_kv_heads != 0) return 0;
+  return nvfp4kv::workspace_layout(num_seqs, num_kv_heads, head_size,
+                                   num_q_heads / num_kv_heads).total;
 }
 
 int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_tokens,

@@ -30,8 +30,8 @@ namespace nvfp4kv {
 size_t decode_smem_bytes(int head_size, int block_size, int num_seqs);
 
 // Largest workspace this entry point can serve (NVFP4_NOALLOC_SCRATCH_BYTES,
-// 12 MiB: head_size 256 needs about 9.8 MiB of partial-result slots plus 4
-// bytes per (sequence, kv head)).
+// 12 MiB): partial-result slots take 4736 * G * head_size * 4 bytes (4.9 MB
+// for G = 2, head_size 128), plus 4 bytes per (sequence, kv head).
 constexpr size_t kNoAllocScratchBytes = NVFP4_NOALLOC_SCRATCH_BYTES;
 }  // namespace nvfp4kv
 
@@ -95,8 +95,8 @@ int nvfp4_paged_attention_noalloc(const void* q, int64_t q_token_stride, int64_t
     return NVFP4_ERR_UNSUPPORTED;
   if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs) > 226 * 1024)
     return NVFP4_ERR_UNSUPPORTED;
-  const nvfp4kv::WorkspaceLayout wl =
-      nvfp4kv::workspace_layout(num_seqs, num_kv_heads, head_size);
+  const nvfp4kv::WorkspaceLayout wl = nvfp4kv::workspace_layout(
+      num_seqs, num_kv_heads, head_size, num_q_heads / num_kv_heads);
   if (wl.total > nvfp4kv::kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;
 
   void* scratch = nullptr;

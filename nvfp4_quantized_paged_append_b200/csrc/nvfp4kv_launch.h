@@ -53,27 +53,31 @@ struct AttentionArgs {
   void* workspace;
 };
 
-// Decode split-KV grid: CTAs launched for the flattened page range. The
-// workspace holds two partial-state slots per CTA.
+// Decode split-KV: at most kDecodeCtas CTAs of 4 warps; every warp owns a
+// contiguous piece of the flattened key range and has two partial-state slots
+// in the workspace.
 constexpr int kDecodeCtas = 148 * 4;
+constexpr int kDecodeWarps = kDecodeCtas * 4;
 
 // Workspace layout (bytes from the start, all 256-byte aligned):
 //   [0, 256)                     uint32 device status word (+ padding)
-//   counters: int32 [num_seqs * num_kv_heads]
-//   partials: float [kDecodeCtas * 2][8 rows][head_size] accumulators
-//   partial m/l: float [kDecodeCtas * 2][8 rows][2]
+//   counters: int32 [num_seqs * num_kv_heads] completion tickets
+//   partials: float [kDecodeWarps * 2][group][head_size] accumulators
+//   partial m/l: float [kDecodeWarps * 2][group][2]
 struct WorkspaceLayout {
   size_t counters_off, partials_off, ml_off, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-__host__ __device__ inline WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads, int head_size) {
+__host__ __device__ inline WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads,
+                                                            int head_size, int group) {
   WorkspaceLayout w;
   w.counters_off = 256;
   w.partials_off = align256(w.counters_off + sizeof(int32_t) * (size_t)num_seqs * num_kv_heads);
-  w.ml_off = align256(w.partials_off + sizeof(float) * (size_t)kDecodeCtas * 2 * 8 * head_size);
-  w.total = align256(w.ml_off + sizeof(float) * (size_t)kDecodeCtas * 2 * 8 * 2);
+  w.ml_off = align256(w.partials_off +
+                      sizeof(float) * (size_t)kDecodeWarps * 2 * group * head_size);
+  w.total = align256(w.ml_off + sizeof(float) * (size_t)kDecodeWarps * 2 * group * 2);
   return w;
 }
 
