@@ -257,39 +257,29 @@ def run_ours(args, rank, world, dist):
         st.append(nk, stream)
         st.attend(nk, stream)
     stream.synchronize()
-    # NG graphs of R = copies steps each; every attention launch in them is
-    # bracketed by its own external (graph-node) timing events, so the kernel's
-    # own device time is measured inside the timed region itself. One-step
-    # graphs serve the K mod R remainder.
-    NG = 4
-    group_graphs, group_events = [], []
-    for g in range(NG):
-        graph = torch.cuda.CUDAGraph()
-        evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(copies)]
-        with torch.cuda.graph(graph, stream=stream):
-            for i, st in enumerate(states):
-                st.append(nk, stream)
-                evs[i][0].record(stream)
-                st.attend(nk, stream)
-                evs[i][1].record(stream)
-        group_graphs.append(graph)
-        group_events.append(evs)
-    single = []
+    # One CUDA graph per kernel per buffer copy. Each timed step replays the
+    # copy's append graph, then its attention graph bracketed by two CUDA
+    # events recorded on the launching stream, so the attention kernel's own
+    # device time is measured inside the timed region itself.
+    g_app, g_att = [], []
     for st in states:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
+        ga = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga, stream=stream):
             st.append(nk, stream)
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb, stream=stream):
             st.attend(nk, stream)
-        single.append(graph)
+        g_app.append(ga)
+        g_att.append(gb)
 
-    def run_steps(n):
-        full, rem = divmod(n, copies)
-        for j in range(full):
-            group_graphs[j % NG].replay()
-        for j in range(rem):
-            single[j].replay()
-        return min(full, NG)
+    def run_steps(n, events=None):
+        for j in range(n):
+            g_app[j % copies].replay()
+            if events is not None:
+                events[j][0].record(stream)
+            g_att[j % copies].replay()
+            if events is not None:
+                events[j][1].record(stream)
 
     run_steps(max(3, args.warmup))
     stream.synchronize()
@@ -300,15 +290,17 @@ def run_ours(args, rank, world, dist):
     # sampled clocks are the loaded ones (extra warm-up, not timed)
     t_end = time.time() + 1.5
     while time.time() < t_end:
-        run_steps(NG * copies * 8)
+        run_steps(200)
         stream.synchronize()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     barrier(dist)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks.mark()
     e0.record(stream)
-    used_groups = run_steps(args.steps)
+    run_steps(args.steps, kev)
     e1.record(stream)
     stream.synchronize()
     clocks.mark()
@@ -318,13 +310,7 @@ def run_ours(args, rank, world, dist):
     ms = max_over_ranks(ms_local, dist)
     ms_step = ms / args.steps
     clocks.stop()
-    # attention kernel durations from the last replay of each group graph
-    kt = [a.elapsed_time(b) for evs in group_events[:used_groups] for a, b in evs]
-    if not kt:  # fewer steps than one group: time one group replay now
-        group_graphs[0].replay()
-        stream.synchronize()
-        kt = [a.elapsed_time(b) for a, b in group_events[0]]
-    attn_ms = statistics.mean(kt)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
 
     # ---- quantize-append sweep (8192 tokens) for Mtok/s
     app = wl.make_append()
@@ -404,7 +390,7 @@ def run_ours(args, rank, world, dist):
             "kv_bytes_per_step": kv_bytes, "new_tokens_per_step": w.num_seqs,
             "l2": f"inputs rotated over {copies} copies ({copies * cache_bytes / 2**20:.0f} MiB of cache) > 4x L2",
             "parallelism": f"replicas x{world} (independent shards, no collective)",
-            "step": "quantize-append of 32 new tokens + decode attention (CUDA graph replay)",
+            "step": "quantize-append of 32 new tokens + decode attention (one CUDA graph per kernel)",
         },
         "roofline": {
             "bound": "hbm", "kernel": "decode_attention_kernel<128,16>",

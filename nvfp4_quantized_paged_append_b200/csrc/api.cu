@@ -6,7 +6,7 @@
 #include "nvfp4kv_launch.h"
 
 namespace nvfp4kv {
-size_t decode_smem_bytes(int head_size, int block_size, int num_seqs);
+size_t decode_smem_bytes(int head_size, int block_size, int num_seqs, int group);
 }
 
 namespace {
@@ -116,7 +116,7 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
   // flattened page indices are int32 on the device
   if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
     return NVFP4_ERR_UNSUPPORTED;
-  if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs) > 226 * 1024)
+  if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) > 226 * 1024)
     return NVFP4_ERR_UNSUPPORTED;
   const size_t need = nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
                                                            head_size);

@@ -43,14 +43,23 @@ namespace nvfp4kv {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;       // units in flight per warp
 constexpr int kUnitTok = 32;     // keys per unit
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;  // lazy max: P stays <= 2^8
 
+// One persistent CTA per SM: all of an SM's warps belong to the same block, so
+// none of them is starved behind an older co-resident block. head_size 256
+// needs more registers and larger pages: fewer warps and stages.
+template <int D>
+struct DecodeCfg {
+  static constexpr int kWarps = (D == 256) ? 8 : 12;
+  static constexpr int kStages = (D == 256) ? 2 : 3;  // units in flight per warp
+};
+
 template <int D, int BS>
 struct DecodeShape {
+  static constexpr int kWarps = DecodeCfg<D>::kWarps;
+  static constexpr int kStages = DecodeCfg<D>::kStages;
   static constexpr int F = D / 2 + D / 16;
   static constexpr int PAGE = BS * F;           // bytes of one (block, K|V, head) page
   static constexpr int U = kUnitTok / BS;       // pages per unit
@@ -89,6 +98,15 @@ __device__ __forceinline__ void write_output(const AttentionArgs& a, int64_t idx
   if (a.o_bf16)
     reinterpret_cast<__nv_bfloat16*>(a.o_bf16)[idx] =
         __float2bfloat16_rn(__fmul_rn(e4m3_to_f32(code), o_scale));
+}
+
+// Read-only global load that stays where it is written (a plain read-only load
+// may be moved next to its first use, which would put its latency back on the
+// critical path).
+__device__ __forceinline__ int ldg_early(const int* p) {
+  int v;
+  asm volatile("ld.global.nc.b32 %0, [%1];\n" : "=r"(v) : "l"(p));
+  return v;
 }
 
 // Locate flattened unit f: advance cursor b so that cum[b] <= f < cum[b+1].
@@ -430,8 +448,10 @@ __device__ __forceinline__ void decode_unit(uint32_t kt0, uint32_t kt1, int vali
 }  // namespace
 
 template <int D, int BS, bool DUP>
-__global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attention_kernel(const AttentionArgs a) {
+__global__ void __launch_bounds__(DecodeCfg<D>::kWarps * 32, 1)
+    decode_attention_kernel(const AttentionArgs a) {
   using S = DecodeShape<D, BS>;
+  constexpr int kWarps = S::kWarps, kStages = S::kStages;
   constexpr int F = S::F, PAGE = S::PAGE, NCH = S::NCH, U = S::U, STAGE = S::STAGE;
   extern __shared__ __align__(128) uint8_t smem[];
   const int Hkv = a.num_kv_heads, G = a.num_q_heads / Hkv;
@@ -508,41 +528,44 @@ __global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attent
   const int nk = e - s;
   bool poisoned = false;
 
-  // issue cursor (all lanes, uniform): segment (ib, ih) spans flattened units
-  // [i_start, i_start + iU); i_pages pages, i_L keys
-  int i_f = s, ib = 0, ih = 0, i_start = 0, iU = 1, i_pages = 1, i_L = 0;
-  auto cursor_seek = [&]() {
-    ib = seek(cum, ib, i_f);
-    iU = (cum[ib + 1] - cum[ib]) / Hkv;
-    ih = (i_f - cum[ib]) / iU;
-    i_start = cum[ib] + ih * iU;
-    i_L = a.seq_lens[ib];
-    i_pages = min(a.max_blocks_per_seq, max(1, (i_L + BS - 1) / BS));
-  };
-  // block ids of the next unit to issue, loaded one step ahead
-  long long nblk[U];
-  int n_pg = 0, n_h = 0, n_L = 0;
-  auto prepare = [&]() {  // cursor -> unit i_f: load its block ids
-    if (i_f >= i_start + iU) cursor_seek();
-    const int u = i_f - i_start;
-    n_pg = min(U, i_pages - u * U);
-    n_h = ih;
-    n_L = i_L;
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      nblk[j] = 0;
-      if (j < n_pg && i_L > 0)
-        nblk[j] = __ldg(a.block_table + (long long)ib * a.max_blocks_per_seq + u * U + j);
+  // Block ids are fetched 32 units at a time, lane j holding unit base + j of
+  // this warp (two banks, refilled a whole batch ahead), so no global load
+  // latency sits between finishing a unit and issuing the copies of the next.
+  int bid0[2] = {0, 0}, bid1[2] = {0, 0}, bmeta[2] = {0, 0};  // meta: h << 8 | n_pg << 1 | keys
+  int l_ib = 0;  // this lane's cursor into cum
+  auto batch_load = [&](int base) {
+    const int bank = (base >> 5) & 1;
+    bid0[bank] = bid1[bank] = bmeta[bank] = 0;
+    const int f = s + base + lane;
+    if (f < e) {
+      l_ib = seek(cum, l_ib, f);
+      const int uu = (cum[l_ib + 1] - cum[l_ib]) / Hkv;
+      const int hh = (f - cum[l_ib]) / uu;
+      const int u = f - cum[l_ib] - hh * uu;
+      const int Lb = a.seq_lens[l_ib];
+      const int pages = min(a.max_blocks_per_seq, max(1, (Lb + BS - 1) / BS));
+      const int npg = min(U, pages - u * U);
+      const int* row = a.block_table + (long long)l_ib * a.max_blocks_per_seq + u * U;
+      if (Lb > 0) {
+        bid0[bank] = ldg_early(row);
+        if (U > 1 && npg > 1) bid1[bank] = ldg_early(row + 1);
+      }
+      bmeta[bank] = (hh << 8) | (npg << 1) | (Lb > 0 ? 1 : 0);
     }
   };
   auto issue = [&](int k) {  // unit k of this warp into stage k % kStages
     const int st = k % kStages;
+    const int bank = (k >> 5) & 1, src = k & 31;
+    const int meta = __shfl_sync(0xffffffffu, bmeta[bank], src);
+    long long blk[2];
+    blk[0] = __shfl_sync(0xffffffffu, bid0[bank], src);
+    blk[1] = __shfl_sync(0xffffffffu, bid1[bank], src);
+    const int n_pg = (meta >> 1) & 0x7F, n_h = meta >> 8;
+    const bool has_keys = meta & 1;
     int okbits = 0;
-    long long blk[U];
 #pragma unroll
     for (int j = 0; j < U; ++j) {
-      blk[j] = nblk[j];
-      if (j < n_pg && n_L > 0) {
+      if (j < n_pg && has_keys) {
         if (blk[j] >= 0 && blk[j] < a.num_blocks) {
           okbits |= 1 << j;
         } else {
@@ -553,9 +576,11 @@ __global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attent
         blk[j] = 0;
       }
     }
+    // The stage being refilled was last read by this warp's own ld.shared
+    // instructions, all complete before the __syncwarp that precedes this
+    // call; the copies only write, so no proxy fence is needed here.
     if (lane == 0) {
       my_ok[st] = okbits;
-      fence_proxy_async_smem();
       mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * n_pg);
 #pragma unroll
       for (int j = 0; j < U; ++j) {
@@ -567,15 +592,12 @@ __global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attent
         }
       }
     }
-    ++i_f;
+    // entering a new batch of 32: fetch the one after it into the other bank
+    if ((k & 31) == 0 && k + 32 < nk) batch_load(k + 32);
   };
 
-  cursor_seek();
-  for (int k = 0; k < min(kStages, nk); ++k) {
-    prepare();
-    issue(k);
-  }
-  if (kStages < nk) prepare();
+  batch_load(0);
+  for (int k = 0; k < min(kStages, nk); ++k) issue(k);
 
   const float k_scale = __ldg(a.kv_scales);
   const float v_scale = __ldg(a.kv_scales + 1);
@@ -683,10 +705,7 @@ __global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attent
                                   acc, g8, t4, PAGE);
       }
       __syncwarp();
-      if (!poisoned && k + kStages < nk) {
-        issue(k + kStages);
-        if (k + kStages + 1 < nk) prepare();
-      }
+      if (!poisoned && k + kStages < nk) issue(k + kStages);
       ++k;
     }
 
@@ -764,65 +783,86 @@ __global__ void __launch_bounds__(kWarps * 32, (D == 256 ? 2 : 3)) decode_attent
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence();
-        // lanes fetch the contributors' (m, l) in parallel (32 at a time)
+        // lane c fetches contributor c's (m, l) for every head (32 at a time)
         const int nc = i_last - i_first + 1;
-        for (int n = 0; n < G; ++n) {
-          float M = -INFINITY;
-          for (int c0 = 0; c0 < nc; c0 += 32) {
-            const int i = i_first + c0 + lane;
-            if (c0 + lane < nc) {
-              const int si = (int)((long long)i * W / n_eff);
-              const size_t ps = (size_t)i * 2 + ((si >= seg_start) ? 0 : 1);
-              M = fmaxf(M, __ldcg(part_ml + (ps * G + n) * 2));
-            }
-          }
+        for (int n0 = 0; n0 < G; n0 += 2) {  // two heads per pass
+          const int nh = min(2, G - n0);
+          float M[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+          float sum[2][D / 32];
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-          const float Mu = (M == -INFINITY) ? 0.0f : M;
-          float lsum = 0.0f;
-          float sum[D / 32];
+          for (int q = 0; q < 2; ++q)
 #pragma unroll
-          for (int j = 0; j < D / 32; ++j) sum[j] = 0.0f;
+            for (int j = 0; j < D / 32; ++j) sum[q][j] = 0.0f;
           for (int c0 = 0; c0 < nc; c0 += 32) {
-            // this lane's contributor: its weight and l
-            const int i = i_first + c0 + lane;
-            float sc = 0.0f, li = 0.0f;
-            size_t ps_mine = 0;
-            if (c0 + lane < nc) {
+            const int cnt = min(32, nc - c0);
+            float mi[2] = {-INFINITY, -INFINITY}, li[2] = {0.f, 0.f};
+            unsigned long long ps_mine = 0;
+            if (lane < cnt) {
+              const int i = i_first + c0 + lane;
               const int si = (int)((long long)i * W / n_eff);
               ps_mine = (size_t)i * 2 + ((si >= seg_start) ? 0 : 1);
-              sc = ex2(__ldcg(part_ml + (ps_mine * G + n) * 2) - Mu);
-              li = __ldcg(part_ml + (ps_mine * G + n) * 2 + 1);
-            }
-            lsum += li * sc;
-            const int cnt = min(32, nc - c0);
-            for (int c = 0; c < cnt; c += 4) {
-              float scv[4], v[4][D / 32];
-              size_t psv[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                scv[q] = __shfl_sync(0xffffffffu, sc, (c + q) & 31);
-                psv[q] = __shfl_sync(0xffffffffu, (unsigned long long)ps_mine, (c + q) & 31);
+              for (int q = 0; q < 2; ++q) {
+                if (q < nh) {
+                  mi[q] = __ldcg(part_ml + (ps_mine * G + n0 + q) * 2);
+                  li[q] = __ldcg(part_ml + (ps_mine * G + n0 + q) * 2 + 1);
+                }
+              }
+            }
+            // rescale what is accumulated so far to the new running max
+            float sc[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              float mx = mi[q];
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+              const float Mn = fmaxf(M[q], mx);
+              const float Mu = (Mn == -INFINITY) ? 0.0f : Mn;
+              const float al = ex2(M[q] - Mu);
+              lsum[q] *= al;
+#pragma unroll
+              for (int j = 0; j < D / 32; ++j) sum[q][j] *= al;
+              M[q] = Mn;
+              sc[q] = ex2(mi[q] - Mu);
+              float lw = li[q] * sc[q];
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+              lsum[q] += lw;
+            }
+            for (int c = 0; c < cnt; c += 4) {
+              float v[4][2][D / 32], scv[4][2];
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const unsigned long long ps = __shfl_sync(0xffffffffu, ps_mine, (c + r) & 31);
+                scv[r][0] = __shfl_sync(0xffffffffu, sc[0], (c + r) & 31);
+                scv[r][1] = __shfl_sync(0xffffffffu, sc[1], (c + r) & 31);
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+#pragma unroll
+                  for (int j = 0; j < D / 32; ++j)
+                    v[r][q][j] = (c + r < cnt && q < nh)
+                                     ? __ldcg(partials + (ps * G + n0 + q) * D + lane + 32 * j)
+                                     : 0.0f;
               }
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
+              for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int j = 0; j < D / 32; ++j)
-                  v[q][j] = (c + q < cnt) ? __ldcg(partials + (psv[q] * G + n) * D + lane + 32 * j)
-                                          : 0.0f;
+                for (int q = 0; q < 2; ++q)
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int j = 0; j < D / 32; ++j) sum[j] += v[q][j] * scv[q];
+                  for (int j = 0; j < D / 32; ++j) sum[q][j] += v[r][q][j] * scv[r][q];
             }
           }
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+          for (int q = 0; q < 2; ++q) {
+            if (q < nh) {
 #pragma unroll
-          for (int j = 0; j < D / 32; ++j) {
-            const int d = lane + 32 * j;
-            const float o = (lsum > 0.0f) ? __fdiv_rn(sum[j], lsum) * v_scale : 0.0f;
-            write_output(a, ((long long)qt * a.num_q_heads + h * G + n) * D + d, o, o_scale);
+              for (int j = 0; j < D / 32; ++j) {
+                const int d = lane + 32 * j;
+                const float o = (lsum[q] > 0.0f) ? __fdiv_rn(sum[q][j], lsum[q]) * v_scale : 0.0f;
+                write_output(a, ((long long)qt * a.num_q_heads + h * G + n0 + q) * D + d, o,
+                             o_scale);
+              }
+            }
           }
         }
         if (lane == 0) counters[b * Hkv + h] = 0;
@@ -843,6 +883,7 @@ struct DeviceFacts {
 template <int D, int BS, bool DUP>
 static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) {
   using S = DecodeShape<D, BS>;
+  constexpr int kWarps = S::kWarps;
   static DeviceFacts facts[64];
   const int G = a.num_q_heads / a.num_kv_heads;
   const size_t smem = S::smem_bytes(a.num_seqs, G);
@@ -875,14 +916,16 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
-size_t decode_smem_bytes(int head_size, int block_size, int num_seqs) {
-  // upper bound over GQA groups (<= 8)
-  if (head_size == 64 && block_size == 16) return DecodeShape<64, 16>::smem_bytes(num_seqs, 8);
-  if (head_size == 64 && block_size == 32) return DecodeShape<64, 32>::smem_bytes(num_seqs, 8);
-  if (head_size == 128 && block_size == 16) return DecodeShape<128, 16>::smem_bytes(num_seqs, 8);
-  if (head_size == 128 && block_size == 32) return DecodeShape<128, 32>::smem_bytes(num_seqs, 8);
-  if (head_size == 256 && block_size == 16) return DecodeShape<256, 16>::smem_bytes(num_seqs, 8);
-  if (head_size == 256 && block_size == 32) return DecodeShape<256, 32>::smem_bytes(num_seqs, 8);
+size_t decode_smem_bytes(int head_size, int block_size, int num_seqs, int group) {
+#define NVFP4_SMEM_CASE(DD, BB) \
+  if (head_size == DD && block_size == BB) return DecodeShape<DD, BB>::smem_bytes(num_seqs, group);
+  NVFP4_SMEM_CASE(64, 16)
+  NVFP4_SMEM_CASE(64, 32)
+  NVFP4_SMEM_CASE(128, 16)
+  NVFP4_SMEM_CASE(128, 32)
+  NVFP4_SMEM_CASE(256, 16)
+  NVFP4_SMEM_CASE(256, 32)
+#undef NVFP4_SMEM_CASE
   return 0;
 }
 

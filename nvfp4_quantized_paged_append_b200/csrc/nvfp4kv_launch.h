@@ -62,7 +62,7 @@ constexpr int kDecodeWarps = kDecodeCtas * 4;
 // Workspace layout (bytes from the start, all 256-byte aligned):
 //   [0, 256)                     uint32 device status word (+ padding)
 //   counters: int32 [num_seqs * num_kv_heads] completion tickets
-//   partials: float [kDecodeWarps * 2][group][head_size] accumulators
+//   partials: float [kDecodeWarps * 2][group][head_size] accumulators (warps of the whole grid)
 //   partial m/l: float [kDecodeWarps * 2][group][2]
 struct WorkspaceLayout {
   size_t counters_off, partials_off, ml_off, total;
