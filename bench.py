@@ -163,25 +163,34 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def kernel_source_sha():
+KERNEL_SOURCES = {
+    "decode_attention_kernel<128,16>": ["attention_decode.cu", "nvfp4kv_device.cuh",
+                                        "nvfp4kv_launch.h"],
+    "quantize_append_kernel<128>": ["writer.cu", "nvfp4kv_device.cuh", "nvfp4kv_launch.h"],
+}
+
+
+def kernel_source_sha(kernel):
+    """Hash of the source files that define a kernel (stale-profile check)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_quantized_paged_append_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key):
-    """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+def profiled_traffic(kernel, workload):
+    """dram bytes (read + write) per launch from the committed ncu summary
+    (profiles/traffic.json), if it was taken on the current kernel sources;
+    else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get(kernel_key)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -369,7 +378,7 @@ def run_ours(args, rank, world, dist):
 
     peak, peak_kind = peaks()
     achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
-    traffic = profiled_traffic("decode_attention_kernel<128,16>@" + WORKLOAD)
+    traffic = profiled_traffic("decode_attention_kernel<128,16>", WORKLOAD)
     result = {
         "metric": METRIC,
         "value": round(world * kv_bytes / (ms_step * 1e-3) / 1e9, 2),
