@@ -415,6 +415,7 @@ def run_ours(args, rank, world, dist):
             "gbs": round(app_bytes / (app_ms * 1e-3) / 1e9, 1),
             "frac": round(app_bytes / (app_ms * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes": app_bytes,
+            "traffic": profiled_traffic("quantize_append_kernel<128>", "append_sweep"),
         },
         "e2e": {
             "value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
