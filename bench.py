@@ -399,10 +399,10 @@ def run_ours(args, rank, world, dist):
             "kv_bytes_per_step": kv_bytes, "new_tokens_per_step": w.num_seqs,
             "l2": f"inputs rotated over {copies} copies ({copies * cache_bytes / 2**20:.0f} MiB of cache) > 4x L2",
             "parallelism": f"replicas x{world} (independent shards, no collective)",
-            "step": "quantize-append of 32 new tokens + decode attention (one CUDA graph per kernel)",
+            "step": "quantize-append of 32 new tokens + decode attention and its split-KV merge (one CUDA graph per op)",
         },
         "roofline": {
-            "bound": "hbm", "kernel": "decode_attention_kernel<128,16>",
+            "bound": "hbm", "kernel": "decode_attention_kernel<128,16> (+ its split-KV merge)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} HBM copy",
             "traffic": traffic, "algorithmic_bytes_per_launch": kv_bytes,
@@ -422,7 +422,7 @@ def run_ours(args, rank, world, dist):
             "ms_per_step": round(e2e_ms, 5),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
         },
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,  # append, decode attention, split-KV merge
         "clocks": clocks.summary(),
     }
     return result

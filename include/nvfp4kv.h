@@ -134,10 +134,12 @@ NVFP4KV_API size_t nvfp4_paged_attention_workspace_size(int32_t num_seqs, int32_
  *   kv_scales       device fp32 [2] = {k_scale, v_scale}.
  *   sm_scale        softmax scale; <= 0 selects 1/sqrt(head_size).
  *   o_fp8           uint8 E4M3 [num_q_tokens][num_q_heads][head_size]:
- *                   E4M3 RNE satfinite(o / o_scale).
+ *                   E4M3 RNE satfinite(o / o_scale), 2-byte aligned.
  *   o_scale         device fp32 scalar (> 0).
- *   o_bf16          optional bf16 output, same shape: bf16(E4M3(o_fp8)*o_scale).
- *   o_f32           optional fp32 output of o before the FP8 cast (testing).
+ *   o_bf16          optional bf16 output, same shape: bf16(E4M3(o_fp8)*o_scale),
+ *                   4-byte aligned.
+ *   o_f32           optional fp32 output of o before the FP8 cast (testing),
+ *                   8-byte aligned. (Adjacent pairs of d are stored together.)
  *   workspace       device scratch of >= nvfp4_paged_attention_workspace_size
  *                   bytes, 256-byte aligned, ZERO-FILLED before its first use;
  *                   every call that completes leaves it ready for the next

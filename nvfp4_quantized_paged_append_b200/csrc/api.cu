@@ -6,7 +6,7 @@
 #include "nvfp4kv_launch.h"
 
 namespace nvfp4kv {
-size_t decode_smem_bytes(int head_size, int block_size, int num_seqs, int group);
+int decode_warps(int head_size, int block_size, int num_seqs, int group);
 }
 
 namespace {
@@ -110,13 +110,13 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
     return NVFP4_ERR_INVALID_ARG;
   if (q_token_stride < (int64_t)num_q_heads * head_size || q_token_stride % 8 != 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(cache, 16) || (o_bf16 && !aligned(o_bf16, 2)) ||
-      (o_f32 && !aligned(o_f32, 4)))
+  if (!aligned(q, 16) || !aligned(cache, 16) || !aligned(o_fp8, 2) ||
+      (o_bf16 && !aligned(o_bf16, 4)) || (o_f32 && !aligned(o_f32, 8)))
     return NVFP4_ERR_INVALID_ARG;
   // flattened page indices are int32 on the device
   if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
     return NVFP4_ERR_UNSUPPORTED;
-  if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) > 226 * 1024)
+  if (nvfp4kv::decode_warps(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) < 1)
     return NVFP4_ERR_UNSUPPORTED;
   const size_t need = nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
                                                            head_size);

@@ -7,20 +7,22 @@
 // head hq, o = softmax(sm_scale * q K^T) V over the sequence's keys, with
 // K = E2M1 * E4M3 * k_scale and V likewise with v_scale.
 //
-// Work decomposition (B200: 148 SMs): a sequence's keys are cut into units of
-// 32 tokens (two 16-token pages, or one 32-token page). The units of all
-// (sequence, kv head) segments are laid end to end and the flattened range is
-// cut into equal contiguous pieces, one per warp of the whole grid, so every
-// warp streams the same number of bytes whatever the length mix. Warps never
-// wait for one another: a segment cut across warps leaves (acc, m, l) partials
-// in the workspace, and the last warp to finish the segment (atomic ticket, no
-// waiting) merges them with the log-sum-exp rule and writes the output.
+// Work decomposition (B200: 148 SMs, one persistent CTA per SM): a sequence's
+// keys are cut into units of 64 tokens (32 for head_size 256). The units of
+// all (sequence, kv head) segments are laid end to end and the flattened range
+// is cut into equal contiguous pieces, one per warp of the whole grid, so
+// every warp streams the same number of bytes whatever the length mix. Warps
+// never wait for one another: a segment cut across warps leaves (acc, m, l)
+// partials in the workspace. When all warps of a block are done, the block
+// takes one arrival ticket per cut segment it holds pieces of (atomic, no
+// waiting); the block whose ticket completes a segment merges the partials
+// with the log-sum-exp rule and writes the output.
 //
 // Each warp runs its own kStages-deep pipeline: one bulk async copy
 // (cp.async.bulk) per K page and per V page of a unit into shared memory,
 // completed on the stage's mbarrier. Pages are contiguous
-// block_size*full_dim bytes in the HND layout. Block ids of the next unit to
-// issue are loaded one unit ahead.
+// block_size*full_dim bytes in the HND layout. Block ids are fetched and
+// checked 32 units ahead, one unit per lane.
 //
 // Math per 16-token tile (all G <= 8 query heads of the kv head at once):
 //   S^T[tok][n] = Khat[tok][:] . q[n][:]     mma.m16n8k16, A = Khat (f16,
@@ -28,11 +30,14 @@
 //                                              cvt e2m1x2->f16x2, times the
 //                                              E4M3 scale; exact), B = q (f16,
 //                                              scaled by a power of two)
-//   online softmax in fp32 (exp2 domain) over the unit's 32 keys, with the
-//   running max moved only when it grows by more than 2^8
+//   online softmax in fp32 (exp2 domain) over the unit's keys; the running
+//   max moves only when a logit exceeds it by more than 2^8, which a lane
+//   detects on its own values (one vote, no reduction, in the common case)
 //   O^T[d][n] += Vhat^T[d][tok] P[tok][n]     mma.m16n8k16, A = Vhat^T built
 //                                              from nibble-transposed bytes,
-//                                              P = f16 hi + f16 lo
+//                                              P = f16 hi + f16 lo moved from
+//                                              the S^T accumulator layout with
+//                                              movmatrix
 // The contraction index of both products is permuted so that each lane's
 // fragments come from contiguous bytes of a row (the same permutation is
 // applied to q, and the PV output rows map back to d on the way out).
@@ -43,35 +48,51 @@ namespace nvfp4kv {
 
 namespace {
 
-constexpr int kUnitTok = 32;     // keys per unit
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;  // lazy max: P stays <= 2^8
+// dynamic shared memory a decode CTA may use (of the 227 KB an SM offers one
+// block, minus the kernel's static shared memory)
+constexpr size_t kDecodeSmemBudget = 226 * 1024;
 
 // One persistent CTA per SM: all of an SM's warps belong to the same block, so
 // none of them is starved behind an older co-resident block. head_size 256
-// needs more registers and larger pages: fewer warps and stages.
+// needs more registers and larger rows: 32-token units and fewer warps.
 template <int D>
 struct DecodeCfg {
-  static constexpr int kWarps = (D == 256) ? 8 : 12;
-  static constexpr int kStages = (D == 256) ? 2 : 3;  // units in flight per warp
+  static constexpr int kUnitTok = (D == 256) ? 32 : 64;
+  static constexpr int kMaxWarps = (D == 256) ? 8 : 12;
+  static constexpr int kStages = (D == 64) ? 3 : 2;  // units in flight per warp
 };
 
 template <int D, int BS>
 struct DecodeShape {
-  static constexpr int kWarps = DecodeCfg<D>::kWarps;
   static constexpr int kStages = DecodeCfg<D>::kStages;
+  static constexpr int UT = DecodeCfg<D>::kUnitTok;  // keys per unit
+  static constexpr int T = UT / 16;                   // 16-token tiles per unit
   static constexpr int F = D / 2 + D / 16;
-  static constexpr int PAGE = BS * F;           // bytes of one (block, K|V, head) page
-  static constexpr int U = kUnitTok / BS;       // pages per unit
-  static constexpr int STAGE = 2 * U * PAGE;    // [K0][V0]([K1][V1]) bytes
-  static constexpr int NCH = D / 16;            // MMA chunks along d
+  static constexpr int PAGE = BS * F;                  // bytes of one (block, K|V, head) page
+  static constexpr int U = UT >= BS ? UT / BS : 1;     // pages per unit
+  static constexpr int STAGE = 2 * UT * F;             // [K0][V0][K1][V1].. bytes
+  static constexpr int NCH = D / 16;                   // MMA chunks along d
   static_assert(PAGE % 16 == 0, "pages must be 16-byte multiples");
-  static size_t smem_bytes(int num_seqs, int group) {
-    return (size_t)kWarps * kStages * STAGE       // ring
-           + 8 * kWarps * kStages                 // mbarriers
-           + 4 * kWarps * kStages                 // per-stage page-ok bits
-           + 4 * (size_t)kWarps * group * D       // per-warp state (hi + lo combined)
-           + 4 * ((size_t)num_seqs + 1);          // unit prefix
+  static_assert(UT % BS == 0, "a unit holds whole pages");
+  static_assert(U <= 4, "at most four pages per unit");
+  // K tile t of a stage (V tile t follows its K tile by PAGE bytes)
+  static constexpr int ktile(int t) { return (16 * t / BS) * 2 * PAGE + ((16 * t) % BS) * F; }
+  // per warp: page ring, query rows of one kv head, kStages + 1 mbarriers,
+  // per-stage page masks
+  static size_t per_warp(int group) {
+    return (size_t)kStages * STAGE + (size_t)group * D * 2 + 8 * (kStages + 1) + 4 * kStages;
+  }
+  // per block: unit prefix, units per kv head, keys and query token per sequence
+  static size_t fixed(int num_seqs) { return 16 * (size_t)num_seqs + 8; }
+  static int warps_for(int num_seqs, int group) {
+    const size_t f = fixed(num_seqs), pw = per_warp(group);
+    if (f + pw > kDecodeSmemBudget) return 0;
+    return (int)std::min<size_t>(DecodeCfg<D>::kMaxWarps, (kDecodeSmemBudget - f) / pw);
+  }
+  static size_t smem_bytes(int num_seqs, int group, int warps) {
+    return warps * per_warp(group) + fixed(num_seqs);
   }
 };
 
@@ -89,15 +110,54 @@ __device__ __forceinline__ float warp_sum_g(float x) {
   return x;
 }
 
-// Final epilogue for one output element.
-__device__ __forceinline__ void write_output(const AttentionArgs& a, int64_t idx, float o,
-                                             float o_scale) {
-  if (a.o_f32) a.o_f32[idx] = o;
-  const uint32_t code = f32_to_e4m3(__fdiv_rn(o, o_scale));
-  a.o_fp8[idx] = (uint8_t)code;
-  if (a.o_bf16)
-    reinterpret_cast<__nv_bfloat16*>(a.o_bf16)[idx] =
-        __float2bfloat16_rn(__fmul_rn(e4m3_to_f32(code), o_scale));
+// Output pointers and scale of the epilogue.
+struct OutPtrs {
+  uint8_t* o_fp8;
+  __nv_bfloat16* o_bf16;  // may be null
+  float* o_f32;           // may be null
+  float inv_os, o_scale;
+};
+
+// Final epilogue for one output element (o already in output units):
+// E4M3(o / o_scale), and optionally fp32 o and bf16(E4M3 * o_scale).
+__device__ __forceinline__ void write_output(const OutPtrs& op, int64_t idx, float o) {
+  if (op.o_f32) op.o_f32[idx] = o;
+  const uint32_t code = f32_to_e4m3(o * op.inv_os);
+  op.o_fp8[idx] = (uint8_t)code;
+  if (op.o_bf16) op.o_bf16[idx] = __float2bfloat16_rn(__fmul_rn(e4m3_to_f32(code), op.o_scale));
+}
+
+// Two adjacent output elements (idx even; the entry point checks that the
+// output pointers are aligned for the pair stores).
+__device__ __forceinline__ void write_output2(const OutPtrs& op, int64_t idx, float o0,
+                                              float o1) {
+  if (op.o_f32) *reinterpret_cast<float2*>(op.o_f32 + idx) = make_float2(o0, o1);
+  const uint32_t codes = f32x2_to_e4m3x2(o0 * op.inv_os, o1 * op.inv_os);
+  *reinterpret_cast<uint16_t*>(op.o_fp8 + idx) = (uint16_t)codes;
+  if (op.o_bf16) {
+    const uint32_t h2 = e4m3x2_to_f16x2(codes);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    *reinterpret_cast<__nv_bfloat162*>(op.o_bf16 + idx) =
+        __floats2bfloat162_rn(__fmul_rn(f.x, op.o_scale), __fmul_rn(f.y, op.o_scale));
+  }
+}
+
+// floor(num / den) for 0 <= num, 0 < den < 2^31 and a quotient below 2^22:
+// a float estimate (approximate reciprocal), corrected by a step or two.
+__device__ __forceinline__ int div_floor(long long num, int den) {
+  float rc;
+  asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(rc) : "f"((float)den));
+  int q = (int)((float)num * rc);
+  long long r = num - (long long)q * den;
+  while (r < 0) {
+    --q;
+    r += den;
+  }
+  while (r >= den) {
+    ++q;
+    r -= den;
+  }
+  return q;
 }
 
 // Read-only global load that stays where it is written (a plain read-only load
@@ -109,10 +169,15 @@ __device__ __forceinline__ int ldg_early(const int* p) {
   return v;
 }
 
-// Locate flattened unit f: advance cursor b so that cum[b] <= f < cum[b+1].
-__device__ __forceinline__ int seek(const int* cum, int b, int f) {
-  while (cum[b + 1] <= f) ++b;
-  return b;
+// The b in [0, n) with cum[b] <= f < cum[b + 1] (cum non-decreasing, cum[0]
+// <= f < cum[n]): binary search over the prefix in shared memory.
+__device__ __forceinline__ int seek_bs(const int* cum, int n, int f) {
+  int lo = 0, hi = n;  // cum[lo] <= f < cum[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cum[mid] <= f) lo = mid; else hi = mid;
+  }
+  return lo;
 }
 
 // Shared-memory loads at a 32-bit shared address.
@@ -188,7 +253,6 @@ __device__ __forceinline__ LaneOffsets lane_offsets(int g8, int t4) {
 template <int D, bool MASK>
 __device__ __forceinline__ void qk_tile(uint32_t kt, const LaneOffsets& lo, int valid, int g8,
                                         const uint32_t (&bq)[D / 16][2], float (&sacc)[4]) {
-  constexpr int NCH = D / 16;
   constexpr int SEG = D / 8;
   uint32_t kw0[SEG / 4], kw1[SEG / 4];
   if constexpr (SEG == 32) {
@@ -269,49 +333,37 @@ __device__ __forceinline__ void qk_tile(uint32_t kt, const LaneOffsets& lo, int 
   }
 }
 
-// P^T of one tile -> B fragments: b0 = P[2t4, 2t4+1][g8], b1 = P[2t4+8, 2t4+9][g8].
-// P = hi + lo (f16 each). DUP (G <= 4): lanes holding the duplicate columns
-// G..2G-1 send lo in place of hi. Otherwise a second fragment carries lo.
+// 8x8 transpose of 16-bit elements across the warp (lane i holds row i/4,
+// columns 2(i%4) and 2(i%4)+1 before and after).
+__device__ __forceinline__ uint32_t movm_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// P^T of one tile (accumulator layout: pr[0..1] = row g8, columns 2t4, 2t4+1;
+// pr[2..3] = row g8+8) -> B fragments b0 = P[2t4, 2t4+1][g8],
+// b1 = P[2t4+8, 2t4+9][g8]. P = hi + lo (f16 each). DUP (G <= 4): the
+// duplicate columns G..2G-1 carry lo in place of hi (lo_sel picks the halves).
+// Otherwise a second fragment pair carries lo.
 template <bool DUP>
-__device__ __forceinline__ void p_fragments(const float (&pr)[4], bool lo0, bool lo1, int g8,
-                                            int t4, uint32_t (&bp)[2], uint32_t (&bpl)[2]) {
-  const uint32_t h_even = pack_f16x2(pr[0], pr[2]);
-  const uint32_t h_odd = pack_f16x2(pr[1], pr[3]);
-  const float2 fe = __half22float2(*reinterpret_cast<const __half2*>(&h_even));
-  const float2 fo = __half22float2(*reinterpret_cast<const __half2*>(&h_odd));
-  const uint32_t l_even = pack_f16x2(pr[0] - fe.x, pr[2] - fe.y);
-  const uint32_t l_odd = pack_f16x2(pr[1] - fo.x, pr[3] - fo.y);
-  const int srcA = (2 * t4) * 4 + (g8 >> 1);
-  const int srcB = srcA + 4;
+__device__ __forceinline__ void p_fragments(const float (&pr)[4], uint32_t lo_sel,
+                                            uint32_t (&bp)[2], uint32_t (&bpl)[2]) {
+  const uint32_t h01 = pack_f16x2(pr[0], pr[1]);
+  const uint32_t h23 = pack_f16x2(pr[2], pr[3]);
+  const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+  const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+  const uint32_t l01 = pack_f16x2(pr[0] - f01.x, pr[1] - f01.y);
+  const uint32_t l23 = pack_f16x2(pr[2] - f23.x, pr[3] - f23.y);
   if constexpr (DUP) {
-    const uint32_t x_even = lo0 ? l_even : h_even;  // column 2t4: rows g8, g8+8
-    const uint32_t x_odd = lo1 ? l_odd : h_odd;     // column 2t4+1
-    const uint32_t ae = __shfl_sync(0xffffffffu, x_even, srcA);
-    const uint32_t ao = __shfl_sync(0xffffffffu, x_odd, srcA);
-    const uint32_t be = __shfl_sync(0xffffffffu, x_even, srcB);
-    const uint32_t bo = __shfl_sync(0xffffffffu, x_odd, srcB);
-    const uint32_t A = (g8 & 1) ? ao : ae;   // (P[2t4][g8], P[2t4+8][g8])
-    const uint32_t Bv = (g8 & 1) ? bo : be;  // (P[2t4+1][g8], P[2t4+9][g8])
-    bp[0] = prmt(A, Bv, 0x5410);
-    bp[1] = prmt(A, Bv, 0x7632);
+    bp[0] = movm_trans(prmt(h01, l01, lo_sel));
+    bp[1] = movm_trans(prmt(h23, l23, lo_sel));
     bpl[0] = bpl[1] = 0u;
   } else {
-    const uint32_t ae = __shfl_sync(0xffffffffu, h_even, srcA);
-    const uint32_t ao = __shfl_sync(0xffffffffu, h_odd, srcA);
-    const uint32_t be = __shfl_sync(0xffffffffu, h_even, srcB);
-    const uint32_t bo = __shfl_sync(0xffffffffu, h_odd, srcB);
-    const uint32_t A = (g8 & 1) ? ao : ae;
-    const uint32_t Bv = (g8 & 1) ? bo : be;
-    bp[0] = prmt(A, Bv, 0x5410);
-    bp[1] = prmt(A, Bv, 0x7632);
-    const uint32_t lae = __shfl_sync(0xffffffffu, l_even, srcA);
-    const uint32_t lao = __shfl_sync(0xffffffffu, l_odd, srcA);
-    const uint32_t lbe = __shfl_sync(0xffffffffu, l_even, srcB);
-    const uint32_t lbo = __shfl_sync(0xffffffffu, l_odd, srcB);
-    const uint32_t LA = (g8 & 1) ? lao : lae;
-    const uint32_t LB = (g8 & 1) ? lbo : lbe;
-    bpl[0] = prmt(LA, LB, 0x5410);
-    bpl[1] = prmt(LA, LB, 0x7632);
+    bp[0] = movm_trans(h01);
+    bp[1] = movm_trans(h23);
+    bpl[0] = movm_trans(l01);
+    bpl[1] = movm_trans(l23);
   }
 }
 
@@ -381,87 +433,189 @@ __device__ __forceinline__ void pv_tile(uint32_t vt, const LaneOffsets& lo, int 
   }
 }
 
-// One 32-token unit: tiles at kt0 and kt1 (V tiles v_off bytes further);
-// tile 1 is skipped when valid1 <= 0 (MASK only).
-template <int D, bool MASK, bool DUP>
-__device__ __forceinline__ void decode_unit(uint32_t kt0, uint32_t kt1, int valid0, int valid1,
-                                            const LaneOffsets& lo, const uint32_t (&bq)[D / 16][2],
-                                            float qmult, bool lo0, bool lo1, float (&m_run)[2],
-                                            float (&l_run)[2], float (&acc)[D / 16][4], int g8,
-                                            int t4, uint32_t v_off) {
-  constexpr int NCH = D / 16;
-  const bool two = !MASK || valid1 > 0;
-  float sa[4] = {0.f, 0.f, 0.f, 0.f};
-  float sb[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  qk_tile<D, MASK>(kt0, lo, valid0, g8, bq, sa);
-  if (two) {
+// One unit of T 16-token tiles in the stage at shared address sbase. MASK:
+// tile t holds valid[t] usable keys (0: skipped).
+template <int D, int BS, bool MASK, bool DUP>
+__device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, const LaneOffsets& lo,
+                                            const uint32_t (&bq)[D / 16][2], float qmult,
+                                            uint32_t lo_sel, float (&m_run)[2], float (&l_run)[2],
+                                            float (&acc)[D / 16][4], int g8, int t4) {
+  using S = DecodeShape<D, BS>;
+  constexpr int T = S::T, NCH = S::NCH;
+  float s[T][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sb[i] = 0.f;
-    qk_tile<D, MASK>(kt1, lo, valid1, g8, bq, sb);
-  }
-  // ---- online softmax over the unit's 32 keys (log2 units, lazy max)
-  float pa[4], pb[4];
-  {
-    const float t0 = warp_max_g(fmaxf(fmaxf(sa[0], sa[2]), fmaxf(sb[0], sb[2]))) * qmult;
-    const float t1 = warp_max_g(fmaxf(fmaxf(sa[1], sa[3]), fmaxf(sb[1], sb[3]))) * qmult;
-    const bool up = (t0 > m_run[0] + kRescaleThresh) || (t1 > m_run[1] + kRescaleThresh);
-    if (__any_sync(0xffffffffu, up)) {
-      const float n0 = fmaxf(m_run[0], t0), n1 = fmaxf(m_run[1], t1);
-      // ex2(-inf) = 0 clears a column seen for the first time (its acc and l are 0)
-      const float al0 = ex2(m_run[0] - (n0 == -INFINITY ? 0.f : n0));
-      const float al1 = ex2(m_run[1] - (n1 == -INFINITY ? 0.f : n1));
-      m_run[0] = n0;
-      m_run[1] = n1;
-      l_run[0] *= al0;
-      l_run[1] *= al1;
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        acc[c][0] *= al0;
-        acc[c][1] *= al1;
-        acc[c][2] *= al0;
-        acc[c][3] *= al1;
-      }
+  for (int t = 0; t < T; ++t) {
+    s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.0f;
+    if (!MASK || valid[t] > 0) {
+      qk_tile<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
+    } else {
+      s[t][0] = s[t][1] = s[t][2] = s[t][3] = -INFINITY;
     }
+  }
+  // ---- online softmax (log2 units). x = s * qmult - m_run; the max moves only
+  // when some x exceeds the threshold (or on the first keys of a column).
+  float x[T][4];
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+  {
     const float mu0 = (m_run[0] == -INFINITY) ? 0.f : m_run[0];
     const float mu1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
-    pa[0] = ex2(fmaf(sa[0], qmult, -mu0));
-    pa[1] = ex2(fmaf(sa[1], qmult, -mu1));
-    pa[2] = ex2(fmaf(sa[2], qmult, -mu0));
-    pa[3] = ex2(fmaf(sa[3], qmult, -mu1));
-    pb[0] = ex2(fmaf(sb[0], qmult, -mu0));
-    pb[1] = ex2(fmaf(sb[1], qmult, -mu1));
-    pb[2] = ex2(fmaf(sb[2], qmult, -mu0));
-    pb[3] = ex2(fmaf(sb[3], qmult, -mu1));
-    l_run[0] += (pa[0] + pa[2]) + (pb[0] + pb[2]);
-    l_run[1] += (pa[1] + pa[3]) + (pb[1] + pb[3]);
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      x[t][0] = fmaf(s[t][0], qmult, -mu0);
+      x[t][1] = fmaf(s[t][1], qmult, -mu1);
+      x[t][2] = fmaf(s[t][2], qmult, -mu0);
+      x[t][3] = fmaf(s[t][3], qmult, -mu1);
+      mx0 = fmaxf(mx0, fmaxf(x[t][0], x[t][2]));
+      mx1 = fmaxf(mx1, fmaxf(x[t][1], x[t][3]));
+    }
   }
-  uint32_t bpa[2], bpla[2];
-  p_fragments<DUP>(pa, lo0, lo1, g8, t4, bpa, bpla);
-  pv_tile<D, MASK, DUP>(kt0 + v_off, lo, valid0, t4, bpa, bpla, acc);
-  if (two) {
-    uint32_t bpb[2], bplb[2];
-    p_fragments<DUP>(pb, lo0, lo1, g8, t4, bpb, bplb);
-    pv_tile<D, MASK, DUP>(kt1 + v_off, lo, valid1, t4, bpb, bplb, acc);
+  const bool up = mx0 > (m_run[0] == -INFINITY ? -INFINITY : kRescaleThresh) ||
+                  mx1 > (m_run[1] == -INFINITY ? -INFINITY : kRescaleThresh);
+  if (__any_sync(0xffffffffu, up)) {
+    float c0 = -INFINITY, c1 = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      c0 = fmaxf(c0, fmaxf(s[t][0], s[t][2]));
+      c1 = fmaxf(c1, fmaxf(s[t][1], s[t][3]));
+    }
+    const float t0 = warp_max_g(c0) * qmult, t1 = warp_max_g(c1) * qmult;
+    const float n0 = fmaxf(m_run[0], t0), n1 = fmaxf(m_run[1], t1);
+    const float nu0 = (n0 == -INFINITY) ? 0.f : n0;
+    const float nu1 = (n1 == -INFINITY) ? 0.f : n1;
+    // ex2(-inf) = 0 clears a column seen for the first time (its acc and l are 0)
+    const float al0 = ex2(m_run[0] - nu0);
+    const float al1 = ex2(m_run[1] - nu1);
+    m_run[0] = n0;
+    m_run[1] = n1;
+    l_run[0] *= al0;
+    l_run[1] *= al1;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      acc[c][0] *= al0;
+      acc[c][1] *= al1;
+      acc[c][2] *= al0;
+      acc[c][3] *= al1;
+    }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      x[t][0] = fmaf(s[t][0], qmult, -nu0);
+      x[t][1] = fmaf(s[t][1], qmult, -nu1);
+      x[t][2] = fmaf(s[t][2], qmult, -nu0);
+      x[t][3] = fmaf(s[t][3], qmult, -nu1);
+    }
   }
+  float p[T][4];
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[t][i] = ex2(x[t][i]);
+    l_run[0] += p[t][0] + p[t][2];
+    l_run[1] += p[t][1] + p[t][3];
+  }
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    if (!MASK || valid[t] > 0) {
+      uint32_t bp[2], bpl[2];
+      p_fragments<DUP>(p[t], lo_sel, bp, bpl);
+      pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::PAGE, lo, MASK ? valid[t] : 16, t4, bp, bpl,
+                            acc);
+    }
+  }
+}
+
+// Merge of one head of a cut segment: its contributors' partials combined
+// with the log-sum-exp rule, then the output. Contributor i (a warp of the
+// decode grid) left (acc, m, l) in slot 0 if the segment is where its piece
+// starts, else in slot 1. Loads of a batch of contributors are all issued
+// before any is used (one round trip to L2 per batch).
+template <int D>
+__device__ __forceinline__ void merge_head(const OutPtrs& op, int num_q_heads,
+                                           const float* partials, const float* part_ml, int G,
+                                           int h, int n, int qt, int i_first, int i_last,
+                                           int seg_start, int W, int n_eff, int lane,
+                                           float v_scale) {
+  constexpr int CH = 8;       // contributors per batch
+  constexpr int J = D / 32;   // elements of d per lane
+  const int nc = i_last - i_first + 1;
+  float M = -INFINITY, lsum = 0.0f;
+  float sum[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) sum[j] = 0.0f;
+  for (int c0 = 0; c0 < nc; c0 += CH) {
+    const int cnt = min(CH, nc - c0);
+    // lane r < cnt: contributor c0 + r's slot and (m, l)
+    unsigned long long ps_mine = 0;
+    float mi = -INFINITY, li = 0.0f;
+    if (lane < cnt) {
+      const int i = i_first + c0 + lane;
+      const int si = div_floor((long long)i * W, n_eff);
+      ps_mine = (unsigned long long)i * 2 + ((si >= seg_start) ? 0 : 1);
+      mi = __ldcg(part_ml + (ps_mine * G + n) * 2);
+      li = __ldcg(part_ml + (ps_mine * G + n) * 2 + 1);
+    }
+    float v[CH][J];
+#pragma unroll
+    for (int r = 0; r < CH; ++r) {
+      const unsigned long long ps = __shfl_sync(0xffffffffu, ps_mine, r);
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+        v[r][j] = (r < cnt) ? __ldcg(partials + (ps * G + n) * D + lane + 32 * j) : 0.0f;
+    }
+    // rescale what is accumulated so far to the new running max
+    float mx = mi;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float Mn = fmaxf(M, mx);
+    const float Mu = (Mn == -INFINITY) ? 0.0f : Mn;
+    const float al = ex2(M - Mu);
+    lsum *= al;
+#pragma unroll
+    for (int j = 0; j < J; ++j) sum[j] *= al;
+    M = Mn;
+    const float sc = ex2(mi - Mu);
+    float lw = li * sc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+    lsum += lw;
+#pragma unroll
+    for (int r = 0; r < CH; ++r) {
+      const float wr = __shfl_sync(0xffffffffu, sc, r);
+#pragma unroll
+      for (int j = 0; j < J; ++j) sum[j] += v[r][j] * wr;
+    }
+  }
+  const float scl = (lsum > 0.0f) ? v_scale / lsum : 0.0f;
+  const long long obase = ((long long)qt * num_q_heads + h * G + n) * D;
+#pragma unroll
+  for (int j = 0; j < J; ++j) write_output(op, obase + lane + 32 * j, sum[j] * scl);
 }
 
 }  // namespace
 
 template <int D, int BS, bool DUP>
-__global__ void __launch_bounds__(DecodeCfg<D>::kWarps * 32, 1)
+__global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
     decode_attention_kernel(const AttentionArgs a) {
   using S = DecodeShape<D, BS>;
-  constexpr int kWarps = S::kWarps, kStages = S::kStages;
-  constexpr int F = S::F, PAGE = S::PAGE, NCH = S::NCH, U = S::U, STAGE = S::STAGE;
+  constexpr int kStages = S::kStages;
+  constexpr int PAGE = S::PAGE, NCH = S::NCH, U = S::U, UT = S::UT, T = S::T;
+  constexpr int STAGE = S::STAGE;
   extern __shared__ __align__(128) uint8_t smem[];
+  const int nw = blockDim.x >> 5;
   const int Hkv = a.num_kv_heads, G = a.num_q_heads / Hkv;
   const int B = a.num_seqs;
+  const int QB = G * D * 2;  // bytes of the query rows of one kv head
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kWarps * kStages * STAGE);
-  int* page_ok = reinterpret_cast<int*>(bars + kWarps * kStages);
-  float* wstate = reinterpret_cast<float*>(page_ok + kWarps * kStages);  // [kWarps][G][D]
-  int* cum = reinterpret_cast<int*>(wstate + kWarps * G * D);
-  __shared__ int warp_tot[kWarps];
+  uint8_t* qbuf = ring + (size_t)nw * kStages * STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + (size_t)nw * QB);  // [nw][kStages + 1]
+  int* stage_ok = reinterpret_cast<int*>(bars + nw * (kStages + 1));
+  int* cum = stage_ok + nw * kStages;  // [B + 1] unit prefix
+  int* sub = cum + B + 1;              // [B] units per kv head
+  int* slen = sub + B;                 // [B] keys
+  int* sqt = slen + B;                 // [B] query token
+  __shared__ int warp_tot[DecodeCfg<D>::kMaxWarps];
+  __shared__ int cut_sg[2 * DecodeCfg<D>::kMaxWarps];  // [warp][slot]: cut segment or -1
+  __shared__ int won[2 * DecodeCfg<D>::kMaxWarps];     // segments this block merges
+  __shared__ int nwon;
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
@@ -470,19 +624,27 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kWarps * 32, 1)
   int* counters = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.counters_off);
   float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.partials_off);
   float* part_ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.ml_off);
+  if (tid < 2 * DecodeCfg<D>::kMaxWarps) cut_sg[tid] = -1;
+  if (tid == 0) nwon = 0;
 
-  // ---- 1. unit prefix over decode sequences (q_len == 1): cum[b]
+  // ---- 1. unit prefix over decode sequences (q_len == 1): a sequence has
+  // ceil(pages / U) units per kv head, with at least one page (an empty
+  // sequence still writes its zero row) and at most what its block table row
+  // maps.
   int carry = 0;
-  for (int base = 0; base < B; base += kWarps * 32) {
+  for (int base = 0; base < B; base += nw * 32) {
     const int b = base + tid;
     int val = 0;
     if (b < B) {
-      const int ql = a.qo_indptr ? a.qo_indptr[b + 1] - a.qo_indptr[b] : 1;
+      const int q0 = a.qo_indptr ? a.qo_indptr[b] : b;
+      const int ql = a.qo_indptr ? a.qo_indptr[b + 1] - q0 : 1;
       const int L = a.seq_lens[b];
-      // pages of the sequence, at least one (an empty sequence still writes
-      // its zero row) and at most the block table's width; then units
       const int pages = min(a.max_blocks_per_seq, max(1, (L + BS - 1) / BS));
-      val = (ql == 1) ? ((pages + U - 1) / U) * Hkv : 0;
+      const int ub = (pages + U - 1) / U;
+      val = (ql == 1) ? ub * Hkv : 0;
+      sub[b] = (ql == 1) ? ub : 0;
+      slen[b] = L;
+      sqt[b] = q0;
     }
     int x = val;
 #pragma unroll
@@ -493,8 +655,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kWarps * 32, 1)
     if (lane == 31) warp_tot[w] = x;
     __syncthreads();
     int before = 0, total = 0;
-#pragma unroll
-    for (int i = 0; i < kWarps; ++i) {
+    for (int i = 0; i < nw; ++i) {
       before += (i < w) ? warp_tot[i] : 0;
       total += warp_tot[i];
     }
@@ -508,368 +669,365 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kWarps * 32, 1)
 
   // ---- 2. this warp's contiguous piece [s, e) of the W flattened units
   const int W = cum[B];
-  const int n_eff = min((int)gridDim.x * kWarps, W);
-  const int gw = blockIdx.x * kWarps + w;
-  if (gw >= n_eff) return;
-  const int s = (int)((long long)gw * W / n_eff);
-  const int e = (int)((long long)(gw + 1) * W / n_eff);
-  auto warp_of = [&](int f) { return (int)(((long long)(f + 1) * n_eff - 1) / W); };
-
-  uint64_t* my_bars = bars + w * kStages;
-  int* my_ok = page_ok + w * kStages;
-  uint8_t* my_ring_p = ring + (size_t)w * kStages * STAGE;
-  const uint32_t my_ring = smem_u32(my_ring_p);
-  float* my_state = wstate + (size_t)w * G * D;
-  if (lane == 0) {
-    for (int st = 0; st < kStages; ++st) mbar_init(&my_bars[st], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-  const int nk = e - s;
-  bool poisoned = false;
-
-  // Block ids are fetched 32 units at a time, lane j holding unit base + j of
-  // this warp (two banks, refilled a whole batch ahead), so no global load
-  // latency sits between finishing a unit and issuing the copies of the next.
-  int bid0[2] = {0, 0}, bid1[2] = {0, 0}, bmeta[2] = {0, 0};  // meta: h << 8 | n_pg << 1 | keys
-  int l_ib = 0;  // this lane's cursor into cum
-  auto batch_load = [&](int base) {
-    const int bank = (base >> 5) & 1;
-    bid0[bank] = bid1[bank] = bmeta[bank] = 0;
-    const int f = s + base + lane;
-    if (f < e) {
-      l_ib = seek(cum, l_ib, f);
-      const int uu = (cum[l_ib + 1] - cum[l_ib]) / Hkv;
-      const int hh = (f - cum[l_ib]) / uu;
-      const int u = f - cum[l_ib] - hh * uu;
-      const int Lb = a.seq_lens[l_ib];
-      const int pages = min(a.max_blocks_per_seq, max(1, (Lb + BS - 1) / BS));
-      const int npg = min(U, pages - u * U);
-      const int* row = a.block_table + (long long)l_ib * a.max_blocks_per_seq + u * U;
-      if (Lb > 0) {
-        bid0[bank] = ldg_early(row);
-        if (U > 1 && npg > 1) bid1[bank] = ldg_early(row + 1);
-      }
-      bmeta[bank] = (hh << 8) | (npg << 1) | (Lb > 0 ? 1 : 0);
-    }
-  };
-  auto issue = [&](int k) {  // unit k of this warp into stage k % kStages
-    const int st = k % kStages;
-    const int bank = (k >> 5) & 1, src = k & 31;
-    const int meta = __shfl_sync(0xffffffffu, bmeta[bank], src);
-    long long blk[2];
-    blk[0] = __shfl_sync(0xffffffffu, bid0[bank], src);
-    blk[1] = __shfl_sync(0xffffffffu, bid1[bank], src);
-    const int n_pg = (meta >> 1) & 0x7F, n_h = meta >> 8;
-    const bool has_keys = meta & 1;
-    int okbits = 0;
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      if (j < n_pg && has_keys) {
-        if (blk[j] >= 0 && blk[j] < a.num_blocks) {
-          okbits |= 1 << j;
-        } else {
-          if (lane == 0) atomicOr(status, kDevBadBlock);
-          blk[j] = 0;  // copy a valid page instead; its rows are masked
-        }
-      } else {
-        blk[j] = 0;
-      }
-    }
-    // The stage being refilled was last read by this warp's own ld.shared
-    // instructions, all complete before the __syncwarp that precedes this
-    // call; the copies only write, so no proxy fence is needed here.
-    if (lane == 0) {
-      my_ok[st] = okbits;
-      mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * n_pg);
-#pragma unroll
-      for (int j = 0; j < U; ++j) {
-        if (j < n_pg) {
-          const uint8_t* kp = a.cache + ((blk[j] * 2) * Hkv + n_h) * (long long)PAGE;
-          uint8_t* dst = my_ring_p + (size_t)st * STAGE + j * 2 * PAGE;
-          bulk_g2s(dst, kp, PAGE, &my_bars[st]);
-          bulk_g2s(dst + PAGE, kp + (long long)Hkv * PAGE, PAGE, &my_bars[st]);
-        }
-      }
-    }
-    // entering a new batch of 32: fetch the one after it into the other bank
-    if ((k & 31) == 0 && k + 32 < nk) batch_load(k + 32);
-  };
-
-  batch_load(0);
-  for (int k = 0; k < min(kStages, nk); ++k) issue(k);
-
-  const float k_scale = __ldg(a.kv_scales);
+  const int n_eff = min((int)gridDim.x * nw, W);
+  // the warp whose piece holds unit f
+  auto warp_of = [&](int f) { return div_floor((long long)(f + 1) * n_eff - 1, W); };
   const float v_scale = __ldg(a.kv_scales + 1);
   const float o_scale = __ldg(a.o_scale);
-  const LaneOffsets lo = lane_offsets<D>(g8, t4);
-  // DUP: columns G..2G-1 of the lanes' B fragments carry lo parts
-  const bool lo0 = DUP && (2 * t4 >= G) && (2 * t4 < 2 * G);
-  const bool lo1 = DUP && (2 * t4 + 1 >= G) && (2 * t4 + 1 < 2 * G);
-
-  int k = 0;  // this warp's unit counter, continuous across portions
-  int seg_f0 = s;
-  int cb = 0;
-  while (seg_f0 < e) {
-    cb = seek(cum, cb, seg_f0);
-    const int b = cb;
-    const int UB = (cum[b + 1] - cum[b]) / Hkv;
-    const int h = (seg_f0 - cum[b]) / UB;
-    const int seg_start = cum[b] + h * UB, seg_end = seg_start + UB;
-    const int pe = min(e, seg_end);
-    const int L = a.seq_lens[b];
-    const int qt = a.qo_indptr ? a.qo_indptr[b] : b;
-
-    // ---- query fragments: lane (g8, t4) holds q[head of column g8][t4*D/4 + i].
-    // DUP: columns G..2G-1 repeat heads 0..G-1 (their P carries the lo part).
-    const int qhead = DUP ? (g8 < 2 * G ? g8 % G : -1) : (g8 < G ? g8 : -1);
-    uint32_t bq[NCH][2];
-    float qmult;
-    {
-      float qv[D / 4];
-      if (qhead >= 0) {
-        const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                    (long long)qt * a.q_token_stride +
-                                    (long long)(h * G + qhead) * D + t4 * (D / 4);
-#pragma unroll
-        for (int i = 0; i < D / 4; i += 8) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + i));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            qv[i + 2 * j] = __uint_as_float(wv[j] << 16);
-            qv[i + 2 * j + 1] = __uint_as_float(wv[j] & 0xFFFF0000u);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < D / 4; ++i) qv[i] = 0.0f;
-      }
-      float mx = 0.0f;
-#pragma unroll
-      for (int i = 0; i < D / 4; ++i) mx = fmaxf(mx, fabsf(qv[i]));
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      // power-of-two scale putting max|q| in [2^14, 2^15): f16 keeps every bf16 bit
-      const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
-      const int sh = min(126, max(-126, 15 - ex));
-      const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
-      const float qds = __uint_as_float((uint32_t)(127 - sh) << 23);
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        bq[c][0] = pack_f16x2(qv[4 * c] * qs, qv[4 * c + 1] * qs);
-        bq[c][1] = pack_f16x2(qv[4 * c + 2] * qs, qv[4 * c + 3] * qs);
-      }
-      qmult = a.sm_scale * k_scale * kLog2e * qds;  // raw MMA units -> log2 units
-    }
-
-    // ---- running state: columns n0 = 2*t4, n1 = 2*t4+1 (lazily moved max)
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.0f, 0.0f};
-    float acc[NCH][4];
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-
-    while (k < nk && s + k < pe) {
-      const int u = s + k - seg_start;
-      const int st = k % kStages;
-      int okbits = 0;
-      if (!poisoned) {
-        if (mbar_wait_bounded(&my_bars[st], (uint32_t)((k / kStages) & 1))) {
-          okbits = my_ok[st];
-        } else {
-          poisoned = true;
-          if (lane == 0) atomicOr(status, kDevTimeout);
-        }
-      }
-      const uint32_t sbase = my_ring + st * STAGE;
-      const int rem = L - u * kUnitTok;
-      // tile t covers keys 16t..16t+15 of the unit; page t (block_size 16) or 0
-      int v0 = min(16, rem), v1 = min(16, rem - 16);
-      if (BS == 16) {
-        if (!(okbits & 1)) v0 = 0;
-        if (!(okbits & 2)) v1 = 0;
-      } else if (!(okbits & 1)) {
-        v0 = v1 = 0;
-      }
-      const uint32_t kt0 = sbase;
-      const uint32_t kt1 = (BS == 16) ? sbase + 2 * PAGE : sbase + 16 * F;
-      if (v0 >= 16 && v1 >= 16) {
-        decode_unit<D, false, DUP>(kt0, kt1, 16, 16, lo, bq, qmult, lo0, lo1, m_run, l_run, acc,
-                                   g8, t4, PAGE);
-      } else if (v0 > 0 || v1 > 0) {
-        // an unusable page next to a usable one: put the usable tile first
-        const bool first = v0 > 0;
-        decode_unit<D, true, DUP>(first ? kt0 : kt1, first ? kt1 : kt0, first ? v0 : v1,
-                                  first ? max(v1, 0) : 0, lo, bq, qmult, lo0, lo1, m_run, l_run,
-                                  acc, g8, t4, PAGE);
-      }
-      __syncwarp();
-      if (!poisoned && k + kStages < nk) issue(k + kStages);
-      ++k;
-    }
-
-    // ---- this warp's state for the segment piece: m per column (uniform over
-    // g8), l summed over the lanes' rows, acc per head in shared memory
-    const float l0 = warp_sum_g(l_run[0]), l1 = warp_sum_g(l_run[1]);
-    {
-      const int n0 = 2 * t4, n1 = 2 * t4 + 1;
-#pragma unroll
-      for (int m = 0; m < NCH; ++m) {  // heads' own (hi) columns first
-        const int d0 = g8 * (D / 8) + 2 * m;
-        if (n0 < G) {
-          my_state[n0 * D + d0] = acc[m][0];
-          my_state[n0 * D + d0 + 1] = acc[m][2];
-        }
-        if (n1 < G) {
-          my_state[n1 * D + d0] = acc[m][1];
-          my_state[n1 * D + d0 + 1] = acc[m][3];
-        }
-      }
-      if constexpr (DUP) {  // then add the lo columns G..2G-1 onto heads 0..G-1
-        __syncwarp();
-#pragma unroll
-        for (int m = 0; m < NCH; ++m) {
-          const int d0 = g8 * (D / 8) + 2 * m;
-          if (n0 >= G && n0 < 2 * G) {
-            my_state[(n0 - G) * D + d0] += acc[m][0];
-            my_state[(n0 - G) * D + d0 + 1] += acc[m][2];
-          }
-          if (n1 >= G && n1 < 2 * G) {
-            my_state[(n1 - G) * D + d0] += acc[m][1];
-            my_state[(n1 - G) * D + d0 + 1] += acc[m][3];
-          }
-        }
-      }
-      __syncwarp();
-    }
-    // m and l of column n live in the lanes with t4 = n / 2 (lane n / 2 has g8 = 0), slot n & 1
-    auto col_ml = [&](int n, float& mm, float& ll) {
-      const int src = n >> 1;
-      const float ma = __shfl_sync(0xffffffffu, m_run[0], src);
-      const float mb = __shfl_sync(0xffffffffu, m_run[1], src);
-      const float la = __shfl_sync(0xffffffffu, l0, src);
-      const float lb = __shfl_sync(0xffffffffu, l1, src);
-      mm = (n & 1) ? mb : ma;
-      ll = (n & 1) ? lb : la;
+  const OutPtrs op{a.o_fp8, reinterpret_cast<__nv_bfloat16*>(a.o_bf16), a.o_f32, 1.0f / o_scale,
+                   o_scale};
+  const int gw = blockIdx.x * nw + w;
+  if (gw < n_eff) {  // (idle warps go straight to the block's merge step)
+    const int s = div_floor((long long)gw * W, n_eff);
+    const int e = div_floor((long long)(gw + 1) * W, n_eff);
+    // (sequence, kv head, first unit of the segment) of flattened unit f
+    auto locate = [&](int f, int& b, int& h, int& seg_start) {
+      b = seek_bs(cum, B, f);
+      const int ub = sub[b];
+      h = div_floor(f - cum[b], ub);
+      seg_start = cum[b] + h * ub;
     };
 
-    const int i_first = warp_of(seg_start), i_last = warp_of(seg_end - 1);
-    const bool whole = (i_first == i_last);
-    const int slot = (s >= seg_start) ? 0 : 1;
-    for (int n = 0; n < G; ++n) {
-      float mm, ll;
-      col_ml(n, mm, ll);
-      if (whole) {
-        const float inv = (ll > 0.0f) ? 1.0f : 0.0f;
-        for (int d = lane; d < D; d += 32) {
-          const float o = inv != 0.0f ? __fdiv_rn(my_state[n * D + d], ll) * v_scale : 0.0f;
-          write_output(a, ((long long)qt * a.num_q_heads + h * G + n) * D + d, o, o_scale);
-        }
-      } else {
-        const size_t ps = (size_t)gw * 2 + slot;
-        for (int d = lane; d < D; d += 32) partials[(ps * G + n) * D + d] = my_state[n * D + d];
-        if (lane == 0) {
-          part_ml[(ps * G + n) * 2 + 0] = mm;
-          part_ml[(ps * G + n) * 2 + 1] = ll;
-        }
-      }
-    }
-    if (!whole) {
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = (atomicAdd(&counters[b * Hkv + h], 1) == i_last - i_first);
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        // lane c fetches contributor c's (m, l) for every head (32 at a time)
-        const int nc = i_last - i_first + 1;
-        for (int n0 = 0; n0 < G; n0 += 2) {  // two heads per pass
-          const int nh = min(2, G - n0);
-          float M[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
-          float sum[2][D / 32];
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int j = 0; j < D / 32; ++j) sum[q][j] = 0.0f;
-          for (int c0 = 0; c0 < nc; c0 += 32) {
-            const int cnt = min(32, nc - c0);
-            float mi[2] = {-INFINITY, -INFINITY}, li[2] = {0.f, 0.f};
-            unsigned long long ps_mine = 0;
-            if (lane < cnt) {
-              const int i = i_first + c0 + lane;
-              const int si = (int)((long long)i * W / n_eff);
-              ps_mine = (size_t)i * 2 + ((si >= seg_start) ? 0 : 1);
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                if (q < nh) {
-                  mi[q] = __ldcg(part_ml + (ps_mine * G + n0 + q) * 2);
-                  li[q] = __ldcg(part_ml + (ps_mine * G + n0 + q) * 2 + 1);
-                }
-              }
-            }
-            // rescale what is accumulated so far to the new running max
-            float sc[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              float mx = mi[q];
-#pragma unroll
-              for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-              const float Mn = fmaxf(M[q], mx);
-              const float Mu = (Mn == -INFINITY) ? 0.0f : Mn;
-              const float al = ex2(M[q] - Mu);
-              lsum[q] *= al;
-#pragma unroll
-              for (int j = 0; j < D / 32; ++j) sum[q][j] *= al;
-              M[q] = Mn;
-              sc[q] = ex2(mi[q] - Mu);
-              float lw = li[q] * sc[q];
-#pragma unroll
-              for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-              lsum[q] += lw;
-            }
-            for (int c = 0; c < cnt; c += 4) {
-              float v[4][2][D / 32], scv[4][2];
-#pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                const unsigned long long ps = __shfl_sync(0xffffffffu, ps_mine, (c + r) & 31);
-                scv[r][0] = __shfl_sync(0xffffffffu, sc[0], (c + r) & 31);
-                scv[r][1] = __shfl_sync(0xffffffffu, sc[1], (c + r) & 31);
-#pragma unroll
-                for (int q = 0; q < 2; ++q)
-#pragma unroll
-                  for (int j = 0; j < D / 32; ++j)
-                    v[r][q][j] = (c + r < cnt && q < nh)
-                                     ? __ldcg(partials + (ps * G + n0 + q) * D + lane + 32 * j)
-                                     : 0.0f;
-              }
-#pragma unroll
-              for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int q = 0; q < 2; ++q)
-#pragma unroll
-                  for (int j = 0; j < D / 32; ++j) sum[q][j] += v[r][q][j] * scv[r][q];
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            if (q < nh) {
-#pragma unroll
-              for (int j = 0; j < D / 32; ++j) {
-                const int d = lane + 32 * j;
-                const float o = (lsum[q] > 0.0f) ? __fdiv_rn(sum[q][j], lsum[q]) * v_scale : 0.0f;
-                write_output(a, ((long long)qt * a.num_q_heads + h * G + n0 + q) * D + d, o,
-                             o_scale);
-              }
-            }
-          }
-        }
-        if (lane == 0) counters[b * Hkv + h] = 0;
-      }
+    const int nk = e - s;
+
+    uint64_t* my_bars = bars + w * (kStages + 1);  // stage barriers, then the query barrier
+    uint64_t* q_bar = my_bars + kStages;
+    int* my_ok = stage_ok + w * kStages;
+    uint8_t* my_ring_p = ring + (size_t)w * kStages * STAGE;
+    uint8_t* my_q = qbuf + (size_t)w * QB;
+    const uint32_t my_ring = smem_u32(my_ring_p);
+    const uint32_t my_q_s = smem_u32(my_q);
+    if (lane == 0) {
+      for (int st = 0; st <= kStages; ++st) mbar_init(&my_bars[st], 1);
+      fence_mbar_init();
     }
     __syncwarp();
-    seg_f0 = pe;
+    // query rows of kv head h of sequence b into this warp's query buffer
+    auto fetch_q = [&](int b, int h) {
+      if (lane == 0) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q) +
+                             ((long long)sqt[b] * a.q_token_stride + (long long)h * G * D) * 2;
+        mbar_arrive_expect_tx(q_bar, QB);
+        bulk_g2s(my_q, src, QB, q_bar);
+      }
+    };
+
+    bool poisoned = false;
+    // Block ids are fetched 32 units at a time, lane j holding unit base + j of
+    // this warp (two banks, refilled a whole batch ahead), so no global load
+    // latency sits between finishing a unit and issuing the copies of the next.
+    // The lane also checks them: a bad id is not copied and its page masked.
+    // (Two named banks selected with conditionals: a bank index into an array
+    // would put the array in local memory.)
+    int bid0[U], bid1[U];
+    int bmeta0 = 0, bmeta1 = 0;  // h << 16 | ok mask << 8 | pages to copy
+  #pragma unroll
+    for (int j = 0; j < U; ++j) bid0[j] = bid1[j] = 0;
+    auto batch_load = [&](int base) {
+      const int bank = (base >> 5) & 1;
+      int ids[U];
+  #pragma unroll
+      for (int j = 0; j < U; ++j) ids[j] = 0;
+      int meta = 0;
+      if (base + lane < nk) {
+        int b, hh, ss;
+        const int f = s + base + lane;
+        locate(f, b, hh, ss);
+        const int u = f - ss;
+        const int Lb = slen[b];
+        const int pages = min(a.max_blocks_per_seq, max(1, (Lb + BS - 1) / BS));
+        const int npg = (Lb > 0) ? min(U, pages - u * U) : 0;
+        const int* row = a.block_table + (long long)b * a.max_blocks_per_seq + u * U;
+        int ok = 0;
+  #pragma unroll
+        for (int j = 0; j < U; ++j) {
+          if (j < npg) {
+            const int x = ldg_early(row + j);
+            if (x >= 0 && x < a.num_blocks) {
+              ids[j] = x;
+              ok |= 1 << j;
+            } else {
+              atomicOr(status, kDevBadBlock);  // skipped below: a copy of block 0, masked
+            }
+          }
+        }
+        meta = (hh << 16) | (ok << 8) | npg;
+      }
+      if (bank) {
+  #pragma unroll
+        for (int j = 0; j < U; ++j) bid1[j] = ids[j];
+        bmeta1 = meta;
+      } else {
+  #pragma unroll
+        for (int j = 0; j < U; ++j) bid0[j] = ids[j];
+        bmeta0 = meta;
+      }
+    };
+    auto issue = [&](int k) {  // unit k of this warp into stage k % kStages
+      const int st = k % kStages;
+      const int bank = (k >> 5) & 1, src = k & 31;
+      const int meta = __shfl_sync(0xffffffffu, bank ? bmeta1 : bmeta0, src);
+      int blk[U];
+  #pragma unroll
+      for (int j = 0; j < U; ++j) blk[j] = __shfl_sync(0xffffffffu, bank ? bid1[j] : bid0[j], src);
+      const int n_pg = meta & 0xFF, n_h = meta >> 16;
+      // The stage being refilled was last read by this warp's own ld.shared
+      // instructions, all complete before the __syncwarp that precedes this
+      // call; the copies only write, so no proxy fence is needed here.
+      if (lane == 0) {
+        my_ok[st] = (meta >> 8) & 0xFF;
+        mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * n_pg);
+  #pragma unroll
+        for (int j = 0; j < U; ++j) {
+          if (j < n_pg) {
+            const uint8_t* kp = a.cache + ((long long)blk[j] * 2 * Hkv + n_h) * PAGE;
+            uint8_t* dst = my_ring_p + (size_t)st * STAGE + j * 2 * PAGE;
+            bulk_g2s(dst, kp, PAGE, &my_bars[st]);
+            bulk_g2s(dst + PAGE, kp + (long long)Hkv * PAGE, PAGE, &my_bars[st]);
+          }
+        }
+      }
+      // entering a new batch of 32: fetch the one after it into the other bank
+      if ((k & 31) == 0 && k + 32 < nk) batch_load(k + 32);
+    };
+
+    batch_load(0);
+    {
+      int b, h, ss;
+      locate(s, b, h, ss);
+      fetch_q(b, h);
+    }
+    for (int k = 0; k < min(kStages, nk); ++k) issue(k);
+
+    const float k_scale = __ldg(a.kv_scales);
+    const LaneOffsets lo = lane_offsets<D>(g8, t4);
+    // DUP: columns G..2G-1 of the lanes' B fragments carry lo parts
+    const bool lo0 = DUP && (2 * t4 >= G) && (2 * t4 < 2 * G);
+    const bool lo1 = DUP && (2 * t4 + 1 >= G) && (2 * t4 + 1 < 2 * G);
+    const uint32_t lo_sel = (lo0 ? 0x0054u : 0x0010u) | (lo1 ? 0x7600u : 0x3200u);
+
+    int k = 0;  // this warp's unit counter, continuous across portions
+    int portion = 0;
+    {
+      const int r_hi = e;
+      int seg_f0 = s;
+      while (seg_f0 < r_hi) {
+        int b, h, seg_start;
+        locate(seg_f0, b, h, seg_start);
+        const int seg_end = seg_start + sub[b];
+        const int pe = min(r_hi, seg_end);
+        const int L = slen[b];
+        const int qt = sqt[b];
+
+        // ---- query fragments from this warp's query buffer: lane (g8, t4)
+        // holds q[head of column g8][t4*D/4 + i]. DUP: columns G..2G-1 repeat
+        // heads 0..G-1 (their P carries the lo part).
+        const int qhead = DUP ? (g8 < 2 * G ? g8 % G : -1) : (g8 < G ? g8 : -1);
+        uint32_t bq[NCH][2];
+        float qmult;
+        {
+          if (!poisoned && !mbar_wait_bounded(q_bar, (uint32_t)(portion & 1))) {
+            poisoned = true;
+            if (lane == 0) atomicOr(status, kDevTimeout);
+          }
+          float qv[D / 4];
+          if (qhead >= 0 && !poisoned) {
+            const uint32_t qa = my_q_s + (uint32_t)(qhead * D + t4 * (D / 4)) * 2;
+  #pragma unroll
+            for (int i = 0; i < D / 4; i += 8) {
+              uint32_t wv[4];
+              lds_words<16>(qa + 2 * i, wv);
+  #pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                qv[i + 2 * j] = __uint_as_float(wv[j] << 16);
+                qv[i + 2 * j + 1] = __uint_as_float(wv[j] & 0xFFFF0000u);
+              }
+            }
+          } else {
+  #pragma unroll
+            for (int i = 0; i < D / 4; ++i) qv[i] = 0.0f;
+          }
+          float mx = 0.0f;
+  #pragma unroll
+          for (int i = 0; i < D / 4; ++i) mx = fmaxf(mx, fabsf(qv[i]));
+  #pragma unroll
+          for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          // power-of-two scale putting max|q| in [2^14, 2^15): f16 keeps every bf16 bit
+          const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
+          const int sh = min(126, max(-126, 15 - ex));
+          const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
+          const float qds = __uint_as_float((uint32_t)(127 - sh) << 23);
+  #pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            bq[c][0] = pack_f16x2(qv[4 * c] * qs, qv[4 * c + 1] * qs);
+            bq[c][1] = pack_f16x2(qv[4 * c + 2] * qs, qv[4 * c + 3] * qs);
+          }
+          qmult = a.sm_scale * k_scale * kLog2e * qds;  // raw MMA units -> log2 units
+        }
+        __syncwarp();
+        {  // the next portion's query rows, while this one runs
+          if (pe < r_hi && !poisoned) {
+            int nb, nh, nss;
+            locate(pe, nb, nh, nss);
+            fetch_q(nb, nh);
+          }
+        }
+
+        // ---- running state: columns n0 = 2*t4, n1 = 2*t4+1 (lazily moved max)
+        float m_run[2] = {-INFINITY, -INFINITY};
+        float l_run[2] = {0.0f, 0.0f};
+        float acc[NCH][4];
+  #pragma unroll
+        for (int c = 0; c < NCH; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+
+        for (int f = seg_f0; f < pe; ++f, ++k) {
+          const int u = f - seg_start;
+          const int st = k % kStages;
+          int okbits = 0;
+          if (!poisoned) {
+            if (mbar_wait_bounded(&my_bars[st], (uint32_t)((k / kStages) & 1))) {
+              okbits = my_ok[st];
+            } else {
+              poisoned = true;
+              if (lane == 0) atomicOr(status, kDevTimeout);
+            }
+          }
+          const uint32_t sbase = my_ring + st * STAGE;
+          const int rem = L - u * UT;  // keys of this unit (clipped per tile below)
+          if (rem >= UT && okbits == (1 << U) - 1) {
+            decode_unit<D, BS, false, DUP>(sbase, nullptr, lo, bq, qmult, lo_sel, m_run, l_run,
+                                           acc, g8, t4);
+          } else {
+            int vv[T];
+            bool any = false;
+  #pragma unroll
+            for (int t = 0; t < T; ++t) {
+              int v = min(16, rem - 16 * t);
+              if (v < 0 || !((okbits >> (16 * t / BS)) & 1)) v = 0;
+              vv[t] = v;
+              any |= v > 0;
+            }
+            if (any)
+              decode_unit<D, BS, true, DUP>(sbase, vv, lo, bq, qmult, lo_sel, m_run, l_run, acc,
+                                            g8, t4);
+          }
+          __syncwarp();
+          if (!poisoned && k + kStages < nk) issue(k + kStages);
+        }
+
+        // ---- this warp's state for the segment piece. l per column summed
+        // over the lanes' rows; DUP: the lo columns G..2G-1 folded onto heads
+        // 0..G-1.
+        const float l0 = warp_sum_g(l_run[0]), l1 = warp_sum_g(l_run[1]);
+        if constexpr (DUP) {
+          if ((G & 1) == 0) {  // column n + G sits G/2 lanes further, same slot
+            const int dl = G >> 1;
+  #pragma unroll
+            for (int m = 0; m < NCH; ++m)
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) acc[m][i] += __shfl_down_sync(0xffffffffu, acc[m][i], dl);
+          } else if (G == 1) {  // column 1 is the lo part of column 0, same lane
+  #pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+              acc[m][0] += acc[m][1];
+              acc[m][2] += acc[m][3];
+            }
+          } else {  // G == 3: column n + 3 lives in lane t4 + (n + 3) / 2 - t4, slot (n + 3) & 1
+            const int c0 = 2 * t4 + G, c1 = 2 * t4 + 1 + G;
+            const int src0 = (lane & ~3) | min(3, c0 >> 1), src1 = (lane & ~3) | min(3, c1 >> 1);
+  #pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+              const float a0 = __shfl_sync(0xffffffffu, acc[m][0], src0);
+              const float a1 = __shfl_sync(0xffffffffu, acc[m][1], src0);
+              const float a2 = __shfl_sync(0xffffffffu, acc[m][2], src0);
+              const float a3 = __shfl_sync(0xffffffffu, acc[m][3], src0);
+              const float b0 = __shfl_sync(0xffffffffu, acc[m][0], src1);
+              const float b1 = __shfl_sync(0xffffffffu, acc[m][1], src1);
+              const float b2 = __shfl_sync(0xffffffffu, acc[m][2], src1);
+              const float b3 = __shfl_sync(0xffffffffu, acc[m][3], src1);
+              acc[m][0] += (c0 & 1) ? a1 : a0;
+              acc[m][2] += (c0 & 1) ? a3 : a2;
+              acc[m][1] += (c1 & 1) ? b1 : b0;
+              acc[m][3] += (c1 & 1) ? b3 : b2;
+            }
+          }
+        }
+
+        const int i_first = warp_of(seg_start), i_last = warp_of(seg_end - 1);
+        const bool whole = (i_first == i_last);
+        const int slot = (s >= seg_start) ? 0 : 1;
+        // column n = 2*t4 + j of this lane: rows d0 = g8*D/8 + 2m and d0 + 1
+        // in acc[m][j] and acc[m][j + 2]
+  #pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int n = 2 * t4 + j;
+          if (n < G) {
+            const float ll = j ? l1 : l0;
+            if (whole) {
+              const float sc = (ll > 0.0f) ? v_scale / ll : 0.0f;
+              const long long obase = ((long long)qt * a.num_q_heads + h * G + n) * D;
+  #pragma unroll
+              for (int m = 0; m < NCH; ++m) {
+                const int d0 = g8 * (D / 8) + 2 * m;
+                write_output2(op, obase + d0, acc[m][j] * sc, acc[m][j + 2] * sc);
+              }
+            } else {
+              const size_t ps = (size_t)gw * 2 + slot;
+              float* dst = partials + (ps * G + n) * D;
+  #pragma unroll
+              for (int m = 0; m < NCH; ++m) {
+                const int d0 = g8 * (D / 8) + 2 * m;
+                *reinterpret_cast<float2*>(dst + d0) = make_float2(acc[m][j], acc[m][j + 2]);
+              }
+              if (g8 == 0) {
+                part_ml[(ps * G + n) * 2 + 0] = m_run[j];
+                part_ml[(ps * G + n) * 2 + 1] = ll;
+              }
+            }
+          }
+        }
+        if (!whole && lane == 0) cut_sg[2 * w + slot] = b * Hkv + h;
+        __syncwarp();
+        seg_f0 = pe;
+        ++portion;
+      }
+    }
+  }  // gw < n_eff
+
+  // ---- 3. cut segments. Every thread's partial writes are made visible
+  // before the block's tickets; the ticket that completes a segment's count
+  // of contributing warps makes this block its merger.
+  __threadfence();
+  __syncthreads();
+  if (tid < 2 * nw) {
+    const int sg = cut_sg[tid];
+    bool first = sg >= 0;
+    int cnt = 0;
+    for (int j = 0; j < 2 * nw; ++j) {
+      if (cut_sg[j] == sg) {
+        ++cnt;
+        if (j < tid) first = false;
+      }
+    }
+    if (first) {
+      const int b = sg / Hkv, h = sg - b * Hkv, ss = cum[b] + h * sub[b];
+      const int nc = warp_of(ss + sub[b] - 1) - warp_of(ss) + 1;
+      if (atomicAdd(&counters[sg], cnt) + cnt == nc) {
+        counters[sg] = 0;  // every contributor has arrived: ready for the next call
+        won[atomicAdd(&nwon, 1)] = sg;
+      }
+    }
+  }
+  __syncthreads();
+  const int n_won = nwon;
+  if (n_won > 0) {
+    __threadfence();
+    for (int t = w; t < n_won * G; t += nw) {  // one (segment, query head) per warp
+      const int sg = won[t / G], n = t % G;
+      const int b = sg / Hkv, h = sg - b * Hkv, ss = cum[b] + h * sub[b];
+      merge_head<D>(op, a.num_q_heads, partials, part_ml, G, h, n, sqt[b], warp_of(ss),
+                    warp_of(ss + sub[b] - 1), ss, W, n_eff, lane, v_scale);
+    }
   }
 }
 
@@ -883,10 +1041,11 @@ struct DeviceFacts {
 template <int D, int BS, bool DUP>
 static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) {
   using S = DecodeShape<D, BS>;
-  constexpr int kWarps = S::kWarps;
   static DeviceFacts facts[64];
   const int G = a.num_q_heads / a.num_kv_heads;
-  const size_t smem = S::smem_bytes(a.num_seqs, G);
+  const int nw = S::warps_for(a.num_seqs, G);
+  if (nw < 1) return cudaErrorInvalidValue;
+  const size_t smem = S::smem_bytes(a.num_seqs, G, nw);
   auto kern = decode_attention_kernel<D, BS, DUP>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -908,24 +1067,24 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
     f.smem_attr_set[DUP] = true;
   }
   int per_sm = 1;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, smem);
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nw * 32, smem);
   if (err != cudaSuccess) return err;
   int grid = f.sms * max(1, per_sm);
-  if (grid > kDecodeCtas) grid = kDecodeCtas;
-  kern<<<grid, kWarps * 32, smem, stream>>>(a);
+  if (grid * nw > kDecodeWarps) grid = kDecodeWarps / nw;
+  kern<<<grid, nw * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-size_t decode_smem_bytes(int head_size, int block_size, int num_seqs, int group) {
-#define NVFP4_SMEM_CASE(DD, BB) \
-  if (head_size == DD && block_size == BB) return DecodeShape<DD, BB>::smem_bytes(num_seqs, group);
-  NVFP4_SMEM_CASE(64, 16)
-  NVFP4_SMEM_CASE(64, 32)
-  NVFP4_SMEM_CASE(128, 16)
-  NVFP4_SMEM_CASE(128, 32)
-  NVFP4_SMEM_CASE(256, 16)
-  NVFP4_SMEM_CASE(256, 32)
-#undef NVFP4_SMEM_CASE
+int decode_warps(int head_size, int block_size, int num_seqs, int group) {
+#define NVFP4_WARPS_CASE(DD, BB) \
+  if (head_size == DD && block_size == BB) return DecodeShape<DD, BB>::warps_for(num_seqs, group);
+  NVFP4_WARPS_CASE(64, 16)
+  NVFP4_WARPS_CASE(64, 32)
+  NVFP4_WARPS_CASE(128, 16)
+  NVFP4_WARPS_CASE(128, 32)
+  NVFP4_WARPS_CASE(256, 16)
+  NVFP4_WARPS_CASE(256, 32)
+#undef NVFP4_WARPS_CASE
   return 0;
 }
 

@@ -27,7 +27,7 @@
 #include "nvfp4kv_launch.h"
 
 namespace nvfp4kv {
-size_t decode_smem_bytes(int head_size, int block_size, int num_seqs, int group);
+int decode_warps(int head_size, int block_size, int num_seqs, int group);
 
 // Largest workspace this entry point can serve (NVFP4_NOALLOC_SCRATCH_BYTES,
 // 12 MiB): partial-result slots take 4736 * G * head_size * 4 bytes (4.9 MB
@@ -88,12 +88,13 @@ int nvfp4_paged_attention_noalloc(const void* q, int64_t q_token_stride, int64_t
   if (q_token_stride < (int64_t)num_q_heads * head_size || q_token_stride % 8 != 0)
     return NVFP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(cache) % 16) ||
-      (o_bf16 && reinterpret_cast<uintptr_t>(o_bf16) % 2) ||
-      (o_f32 && reinterpret_cast<uintptr_t>(o_f32) % 4))
+      (reinterpret_cast<uintptr_t>(o_fp8) % 2) ||
+      (o_bf16 && reinterpret_cast<uintptr_t>(o_bf16) % 4) ||
+      (o_f32 && reinterpret_cast<uintptr_t>(o_f32) % 8))
     return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
     return NVFP4_ERR_UNSUPPORTED;
-  if (nvfp4kv::decode_smem_bytes(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) > 226 * 1024)
+  if (nvfp4kv::decode_warps(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) < 1)
     return NVFP4_ERR_UNSUPPORTED;
   const nvfp4kv::WorkspaceLayout wl = nvfp4kv::workspace_layout(
       num_seqs, num_kv_heads, head_size, num_q_heads / num_kv_heads);

@@ -53,16 +53,18 @@ struct AttentionArgs {
   void* workspace;
 };
 
-// Decode split-KV: at most kDecodeCtas CTAs of 4 warps; every warp owns a
-// contiguous piece of the flattened key range and has two partial-state slots
-// in the workspace.
+// Decode split-KV: at most kDecodeWarps warps in the whole grid; every warp
+// owns a contiguous piece of the flattened key range and has two
+// partial-state slots in the workspace (the segment holding its first unit,
+// and the one holding its last).
 constexpr int kDecodeCtas = 148 * 4;
 constexpr int kDecodeWarps = kDecodeCtas * 4;
 
 // Workspace layout (bytes from the start, all 256-byte aligned):
-//   [0, 256)                     uint32 device status word (+ padding)
-//   counters: int32 [num_seqs * num_kv_heads] completion tickets
-//   partials: float [kDecodeWarps * 2][group][head_size] accumulators (warps of the whole grid)
+//   [0, 256)   uint32 device status word (+ padding)
+//   counters:  int32 [num_seqs * num_kv_heads] arrival counts of the blocks
+//              that hold pieces of a cut segment (back to 0 after each call)
+//   partials:  float [kDecodeWarps * 2][group][head_size] accumulators
 //   partial m/l: float [kDecodeWarps * 2][group][2]
 struct WorkspaceLayout {
   size_t counters_off, partials_off, ml_off, total;

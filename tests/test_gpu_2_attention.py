@@ -111,9 +111,11 @@ def test_repeat_calls_identical_and_workspace_reusable():
     torch.cuda.synchronize()
     for o8, o32 in outs[1:]:
         assert torch.equal(o8, outs[0][0]) and torch.equal(o32, outs[0][1])
-    # counters are back to zero
-    lay_counters = ws[256: 256 + 4 * w.num_seqs * w.num_kv_heads].view(torch.int32)
-    assert int(lay_counters.abs().sum()) == 0
+    # no status bit was raised, and the arrival counters of the cut segments
+    # are back to zero for the next call
+    assert nk.workspace_status(ws) == 0
+    counters = ws[256: 256 + 4 * w.num_seqs * w.num_kv_heads].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
 
 
 def test_bad_block_id_flagged_no_fault():

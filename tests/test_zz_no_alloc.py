@@ -60,17 +60,17 @@ def test_noalloc_matches_workspace_entry_point(make):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    """30000 sequences x 128 kv heads need ~17 MB of workspace (completion
-    tickets + partial slots), more than the fixed 12 MiB array: the call must
-    fail with NVFP4_ERR_WORKSPACE before launching anything. The buffers are
-    real and valid anyway."""
-    B, H, D = 30000, 128, 64
-    assert nk.workspace_size(B, H, H, D) > 12 << 20
-    q = torch.zeros((B, H, D), dtype=torch.bfloat16, device=DEV)
-    cache = nk.alloc_kv_cache(1, 16, H, D, DEV)
+    """64 query heads over 8 kv heads at head_size 256 need ~39 MB of split-KV
+    partial slots, more than the fixed 12 MiB array: the call must fail with
+    NVFP4_ERR_WORKSPACE before launching anything. The buffers are real and
+    valid anyway."""
+    B, HQ, HKV, D = 4, 64, 8, 256
+    assert nk.workspace_size(B, HQ, HKV, D) > 12 << 20
+    q = torch.zeros((B, HQ, D), dtype=torch.bfloat16, device=DEV)
+    cache = nk.alloc_kv_cache(1, 16, HKV, D, DEV)
     bt = torch.zeros((B, 1), dtype=torch.int32, device=DEV)
     sl = torch.ones(B, dtype=torch.int32, device=DEV)
-    o8 = torch.empty((B, H, D), dtype=torch.uint8, device=DEV)
+    o8 = torch.empty((B, HQ, D), dtype=torch.uint8, device=DEV)
     with pytest.raises(nk.Nvfp4Error) as e:
         nk.paged_attention_noalloc(q, cache, bt, sl, torch.ones(2, device=DEV), o8,
                                    torch.ones(1, device=DEV))
