@@ -113,8 +113,9 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
   if (!aligned(q, 16) || !aligned(cache, 16) || !aligned(o_fp8, 2) ||
       (o_bf16 && !aligned(o_bf16, 4)) || (o_f32 && !aligned(o_f32, 8)))
     return NVFP4_ERR_INVALID_ARG;
-  // flattened page indices are int32 on the device
-  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
+  // flattened page indices and cache page rows are int32 on the device
+  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30 ||
+      num_blocks * 2 * num_kv_heads >= (int64_t)1 << 31)
     return NVFP4_ERR_UNSUPPORTED;
   if (nvfp4kv::decode_warps(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) < 1)
     return NVFP4_ERR_UNSUPPORTED;

@@ -44,6 +44,8 @@
 #include "nvfp4kv_device.cuh"
 #include "nvfp4kv_launch.h"
 
+#include <cudaTypedefs.h>
+
 namespace nvfp4kv {
 
 namespace {
@@ -78,7 +80,12 @@ struct DecodeShape {
   static_assert(UT % BS == 0, "a unit holds whole pages");
   static_assert(U <= 4, "at most four pages per unit");
   // K tile t of a stage (V tile t follows its K tile by PAGE bytes)
-  static constexpr int ktile(int t) { return (16 * t / BS) * 2 * PAGE + ((16 * t) % BS) * F; }
+  // stage layout: the unit's K pages, then its V pages
+  static constexpr int ktile(int t) { return (16 * t / BS) * PAGE + ((16 * t) % BS) * F; }
+  static constexpr int VOFF = U * PAGE;  // V tile t = K tile t + VOFF
+  // a unit's pages in one or two gather4 tensor copies (4 rows of one page
+  // each) when a page fits one box row (<= 256 eight-byte elements)
+  static constexpr bool kGather = (U == 2 || U == 4) && PAGE / 8 <= 256;
   // per warp: page ring, query rows of one kv head, kStages + 1 mbarriers,
   // per-stage page masks
   static size_t per_warp(int group) {
@@ -517,7 +524,7 @@ __device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, co
     if (!MASK || valid[t] > 0) {
       uint32_t bp[2], bpl[2];
       p_fragments<DUP>(p[t], lo_sel, bp, bpl);
-      pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::PAGE, lo, MASK ? valid[t] : 16, t4, bp, bpl,
+      pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp, bpl,
                             acc);
     }
   }
@@ -594,7 +601,7 @@ __device__ __forceinline__ void merge_head(const OutPtrs& op, int num_q_heads,
 
 template <int D, int BS, bool DUP>
 __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
-    decode_attention_kernel(const AttentionArgs a) {
+    decode_attention_kernel(const __grid_constant__ AttentionArgs a) {
   using S = DecodeShape<D, BS>;
   constexpr int kStages = S::kStages;
   constexpr int PAGE = S::PAGE, NCH = S::NCH, U = S::U, UT = S::UT, T = S::T;
@@ -721,12 +728,12 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
     // would put the array in local memory.)
     int bid0[U], bid1[U];
     int bmeta0 = 0, bmeta1 = 0;  // h << 16 | ok mask << 8 | pages to copy
-  #pragma unroll
+#pragma unroll
     for (int j = 0; j < U; ++j) bid0[j] = bid1[j] = 0;
     auto batch_load = [&](int base) {
       const int bank = (base >> 5) & 1;
       int ids[U];
-  #pragma unroll
+#pragma unroll
       for (int j = 0; j < U; ++j) ids[j] = 0;
       int meta = 0;
       if (base + lane < nk) {
@@ -739,7 +746,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         const int npg = (Lb > 0) ? min(U, pages - u * U) : 0;
         const int* row = a.block_table + (long long)b * a.max_blocks_per_seq + u * U;
         int ok = 0;
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < U; ++j) {
           if (j < npg) {
             const int x = ldg_early(row + j);
@@ -754,11 +761,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         meta = (hh << 16) | (ok << 8) | npg;
       }
       if (bank) {
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < U; ++j) bid1[j] = ids[j];
         bmeta1 = meta;
       } else {
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < U; ++j) bid0[j] = ids[j];
         bmeta0 = meta;
       }
@@ -768,7 +775,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
       const int bank = (k >> 5) & 1, src = k & 31;
       const int meta = __shfl_sync(0xffffffffu, bank ? bmeta1 : bmeta0, src);
       int blk[U];
-  #pragma unroll
+#pragma unroll
       for (int j = 0; j < U; ++j) blk[j] = __shfl_sync(0xffffffffu, bank ? bid1[j] : bid0[j], src);
       const int n_pg = meta & 0xFF, n_h = meta >> 16;
       // The stage being refilled was last read by this warp's own ld.shared
@@ -777,13 +784,29 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
       if (lane == 0) {
         my_ok[st] = (meta >> 8) & 0xFF;
         mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * n_pg);
-  #pragma unroll
-        for (int j = 0; j < U; ++j) {
-          if (j < n_pg) {
-            const uint8_t* kp = a.cache + ((long long)blk[j] * 2 * Hkv + n_h) * PAGE;
-            uint8_t* dst = my_ring_p + (size_t)st * STAGE + j * 2 * PAGE;
-            bulk_g2s(dst, kp, PAGE, &my_bars[st]);
-            bulk_g2s(dst + PAGE, kp + (long long)Hkv * PAGE, PAGE, &my_bars[st]);
+        uint8_t* dst = my_ring_p + (size_t)st * STAGE;
+        // page row r of the cache: (block, K|V, head) = (r / 2Hkv, r / Hkv % 2, r % Hkv)
+        if (S::kGather && n_pg == U) {
+          const uint32_t d = smem_u32(dst);
+          if constexpr (U == 4) {
+            tma_gather4(d, &a.kv_pages, blk[0] * 2 * Hkv + n_h, blk[1] * 2 * Hkv + n_h,
+                        blk[2] * 2 * Hkv + n_h, blk[3] * 2 * Hkv + n_h, &my_bars[st]);
+            tma_gather4(d + 4 * PAGE, &a.kv_pages, (blk[0] * 2 + 1) * Hkv + n_h,
+                        (blk[1] * 2 + 1) * Hkv + n_h, (blk[2] * 2 + 1) * Hkv + n_h,
+                        (blk[3] * 2 + 1) * Hkv + n_h, &my_bars[st]);
+          } else {
+            tma_gather4(d, &a.kv_pages, blk[0] * 2 * Hkv + n_h, blk[U - 1] * 2 * Hkv + n_h,
+                        (blk[0] * 2 + 1) * Hkv + n_h, (blk[U - 1] * 2 + 1) * Hkv + n_h,
+                        &my_bars[st]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < U; ++j) {
+            if (j < n_pg) {
+              const uint8_t* kp = a.cache + ((long long)blk[j] * 2 * Hkv + n_h) * PAGE;
+              bulk_g2s(dst + j * PAGE, kp, PAGE, &my_bars[st]);
+              bulk_g2s(dst + (U + j) * PAGE, kp + (long long)Hkv * PAGE, PAGE, &my_bars[st]);
+            }
           }
         }
       }
@@ -833,31 +856,31 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
           float qv[D / 4];
           if (qhead >= 0 && !poisoned) {
             const uint32_t qa = my_q_s + (uint32_t)(qhead * D + t4 * (D / 4)) * 2;
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < D / 4; i += 8) {
               uint32_t wv[4];
               lds_words<16>(qa + 2 * i, wv);
-  #pragma unroll
+#pragma unroll
               for (int j = 0; j < 4; ++j) {
                 qv[i + 2 * j] = __uint_as_float(wv[j] << 16);
                 qv[i + 2 * j + 1] = __uint_as_float(wv[j] & 0xFFFF0000u);
               }
             }
           } else {
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < D / 4; ++i) qv[i] = 0.0f;
           }
           float mx = 0.0f;
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < D / 4; ++i) mx = fmaxf(mx, fabsf(qv[i]));
-  #pragma unroll
+#pragma unroll
           for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           // power-of-two scale putting max|q| in [2^14, 2^15): f16 keeps every bf16 bit
           const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
           const int sh = min(126, max(-126, 15 - ex));
           const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
           const float qds = __uint_as_float((uint32_t)(127 - sh) << 23);
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < NCH; ++c) {
             bq[c][0] = pack_f16x2(qv[4 * c] * qs, qv[4 * c + 1] * qs);
             bq[c][1] = pack_f16x2(qv[4 * c + 2] * qs, qv[4 * c + 3] * qs);
@@ -877,7 +900,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         float m_run[2] = {-INFINITY, -INFINITY};
         float l_run[2] = {0.0f, 0.0f};
         float acc[NCH][4];
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < NCH; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
 
         for (int f = seg_f0; f < pe; ++f, ++k) {
@@ -900,7 +923,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
           } else {
             int vv[T];
             bool any = false;
-  #pragma unroll
+#pragma unroll
             for (int t = 0; t < T; ++t) {
               int v = min(16, rem - 16 * t);
               if (v < 0 || !((okbits >> (16 * t / BS)) & 1)) v = 0;
@@ -922,12 +945,12 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         if constexpr (DUP) {
           if ((G & 1) == 0) {  // column n + G sits G/2 lanes further, same slot
             const int dl = G >> 1;
-  #pragma unroll
+#pragma unroll
             for (int m = 0; m < NCH; ++m)
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 4; ++i) acc[m][i] += __shfl_down_sync(0xffffffffu, acc[m][i], dl);
           } else if (G == 1) {  // column 1 is the lo part of column 0, same lane
-  #pragma unroll
+#pragma unroll
             for (int m = 0; m < NCH; ++m) {
               acc[m][0] += acc[m][1];
               acc[m][2] += acc[m][3];
@@ -935,7 +958,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
           } else {  // G == 3: column n + 3 lives in lane t4 + (n + 3) / 2 - t4, slot (n + 3) & 1
             const int c0 = 2 * t4 + G, c1 = 2 * t4 + 1 + G;
             const int src0 = (lane & ~3) | min(3, c0 >> 1), src1 = (lane & ~3) | min(3, c1 >> 1);
-  #pragma unroll
+#pragma unroll
             for (int m = 0; m < NCH; ++m) {
               const float a0 = __shfl_sync(0xffffffffu, acc[m][0], src0);
               const float a1 = __shfl_sync(0xffffffffu, acc[m][1], src0);
@@ -958,7 +981,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         const int slot = (s >= seg_start) ? 0 : 1;
         // column n = 2*t4 + j of this lane: rows d0 = g8*D/8 + 2m and d0 + 1
         // in acc[m][j] and acc[m][j + 2]
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int n = 2 * t4 + j;
           if (n < G) {
@@ -966,7 +989,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
             if (whole) {
               const float sc = (ll > 0.0f) ? v_scale / ll : 0.0f;
               const long long obase = ((long long)qt * a.num_q_heads + h * G + n) * D;
-  #pragma unroll
+#pragma unroll
               for (int m = 0; m < NCH; ++m) {
                 const int d0 = g8 * (D / 8) + 2 * m;
                 write_output2(op, obase + d0, acc[m][j] * sc, acc[m][j + 2] * sc);
@@ -974,7 +997,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
             } else {
               const size_t ps = (size_t)gw * 2 + slot;
               float* dst = partials + (ps * G + n) * D;
-  #pragma unroll
+#pragma unroll
               for (int m = 0; m < NCH; ++m) {
                 const int d0 = g8 * (D / 8) + 2 * m;
                 *reinterpret_cast<float2*>(dst + d0) = make_float2(acc[m][j], acc[m][j + 2]);
@@ -1031,6 +1054,38 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   }
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// The cache as rows of pages: row r is the (block r / 2Hkv, K|V, head) page of
+// `page_bytes` bytes, seen as eight-byte elements; one row per box.
+static cudaError_t encode_page_rows(CUtensorMap* map, const uint8_t* cache, int64_t num_blocks,
+                                    int num_kv_heads, int page_bytes) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)page_bytes / 8,
+                              (cuuint64_t)num_blocks * 2 * num_kv_heads};
+  const cuuint64_t strides[1] = {(cuuint64_t)page_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)page_bytes / 8, 1};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(cache),
+                         dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Per-device launch facts, looked up once (outside any stream capture: the
 // first call on a device should be an eager one).
 struct DeviceFacts {
@@ -1071,7 +1126,14 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   if (err != cudaSuccess) return err;
   int grid = f.sms * max(1, per_sm);
   if (grid * nw > kDecodeWarps) grid = kDecodeWarps / nw;
-  kern<<<grid, nw * 32, smem, stream>>>(a);
+  if constexpr (S::kGather) {
+    AttentionArgs ag = a;
+    err = encode_page_rows(&ag.kv_pages, a.cache, a.num_blocks, a.num_kv_heads, S::PAGE);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, nw * 32, smem, stream>>>(ag);
+  } else {
+    kern<<<grid, nw * 32, smem, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -92,7 +92,8 @@ int nvfp4_paged_attention_noalloc(const void* q, int64_t q_token_stride, int64_t
       (o_bf16 && reinterpret_cast<uintptr_t>(o_bf16) % 4) ||
       (o_f32 && reinterpret_cast<uintptr_t>(o_f32) % 8))
     return NVFP4_ERR_INVALID_ARG;
-  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30)
+  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30 ||
+      num_blocks * 2 * num_kv_heads >= (int64_t)1 << 31)
     return NVFP4_ERR_UNSUPPORTED;
   if (nvfp4kv::decode_warps(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) < 1)
     return NVFP4_ERR_UNSUPPORTED;

@@ -2,6 +2,7 @@
 // Arguments arrive here already validated.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -33,6 +34,10 @@ struct DequantArgs {
 };
 
 struct AttentionArgs {
+  // the cache as a 2-D tensor of page rows (row r = (block, K|V, head) page,
+  // PAGE / 8 eight-byte elements), for gather4 page loads; encoded by the
+  // launcher when the configuration uses them
+  CUtensorMap kv_pages;
   const void* q;
   int64_t q_token_stride, num_q_tokens;
   int num_q_heads;
