@@ -624,6 +624,10 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   __shared__ int won[2 * DecodeCfg<D>::kMaxWarps];     // segments this block merges
   __shared__ int nwon;
 
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (when that kernel allows it): the block may be resident early, but reads
+  // nothing before that kernel has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   uint32_t* status = reinterpret_cast<uint32_t*>(a.workspace);
@@ -1126,14 +1130,25 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   if (err != cudaSuccess) return err;
   int grid = f.sms * max(1, per_sm);
   if (grid * nw > kDecodeWarps) grid = kDecodeWarps / nw;
+  AttentionArgs ag = a;
   if constexpr (S::kGather) {
-    AttentionArgs ag = a;
     err = encode_page_rows(&ag.kv_pages, a.cache, a.num_blocks, a.num_kv_heads, S::PAGE);
     if (err != cudaSuccess) return err;
-    kern<<<grid, nw * 32, smem, stream>>>(ag);
-  } else {
-    kern<<<grid, nw * 32, smem, stream>>>(a);
   }
+  // programmatic dependent launch: the grid may be scheduled while the
+  // previous kernel on the stream finishes (its blocks wait on entry)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)(nw * 32));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, ag);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -55,6 +55,9 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
     uint32_t* __restrict__ status) {
   constexpr int TPR = D / 8;  // threads per row
   constexpr int F = D / 2 + D / 16;
+  // a kernel launched after this one as a programmatic dependent (attention)
+  // may be scheduled now; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int64_t t = blockIdx.x;
   const int64_t slot = __ldg(slot_mapping + t);
   if (slot < 0) return;
