@@ -9,9 +9,8 @@
 // Dequant: "FlashInfer NVFP4 KV serving on pre-SM100 GPUs", quick answer (the
 // paged NVFP4 dequantize helper).
 //
-// Mapping: one CTA per token, one thread per 8 consecutive elements of a row
-// (one 16-byte bf16 load, one 4-byte packed store); the two threads of a
-// 16-element group meet with one shuffle for the block amax.
+// Mapping: one CTA per token, one thread per 16-element block of a row (two
+// 16-byte bf16 loads, one E4M3 scale byte, 8 bytes of packed codes).
 #include "nvfp4kv_device.cuh"
 #include "nvfp4kv_launch.h"
 
@@ -44,8 +43,25 @@ __device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S)
   return f32x8_to_e2m1x8(q);
 }
 
-// One CTA per new token: its K and V rows of every kv head, one thread per 8
-// elements. A skipped (slot < 0) or out-of-range token exits as a whole.
+// E4M3 byte of fl32(a / b) (RNE, satfinite). Fast path as for the codes: the
+// quotient from the approximate reciprocal is within 2^-21 of fl32(a / b);
+// when both ends of the +-2^-20 bracket encode to the same byte, so does
+// fl32(a / b). Otherwise, and for b outside [2^-100, 2^100] or a non-finite
+// a, the quotient is formed with IEEE division.
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float b) {
+  if (b >= 7.8886091e-31f && b <= 1.2676506e30f && a <= 3.4028235e38f) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(b));
+    const float y = a * r;
+    const uint32_t two = f32x2_to_e4m3x2(y * 0.99999904632568359375f, y * 1.00000095367431640625f);
+    if ((two & 0xFFu) == (two >> 8)) return two & 0xFFu;
+  }
+  return f32_to_e4m3(__fdiv_rn(a, b));
+}
+
+// One CTA per new token: its K and V rows of every kv head, one thread per
+// 16-element block (two 16-byte bf16 loads, one scale, 8 bytes of codes). A
+// skipped (slot < 0) or out-of-range token exits as a whole.
 template <int D>
 __global__ void __launch_bounds__(256) quantize_append_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -53,7 +69,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
     int64_t num_blocks, int bs_log2, const int64_t* __restrict__ slot_mapping,
     const float* __restrict__ k_scale, const float* __restrict__ v_scale,
     uint32_t* __restrict__ status) {
-  constexpr int TPR = D / 8;  // threads per row
+  constexpr int TPR = D / 16;  // threads per row
   constexpr int F = D / 2 + D / 16;
   // a kernel launched after this one as a programmatic dependent (attention)
   // may be scheduled now; it waits for this grid's completion before reading
@@ -68,51 +84,51 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
   const int64_t blk = slot >> bs_log2;
   const int off = (int)(slot & ((1 << bs_log2) - 1));
   const int block_size = 1 << bs_log2;
+  const float gk = __ldg(k_scale), gv = __ldg(v_scale);
   const int nthr = 2 * num_kv_heads * TPR;
-  const int nthr_w = (nthr + 31) & ~31;  // whole warps iterate together (pair shuffles)
-  for (int idx = threadIdx.x; idx < nthr_w; idx += blockDim.x) {
-    const bool act = idx < nthr;
+  for (int idx = threadIdx.x; idx < nthr; idx += blockDim.x) {
     const int rr = idx / TPR, j = idx % TPR;
     const int kv = rr >= num_kv_heads ? 1 : 0;
     const int h = rr - kv * num_kv_heads;
-    float x[8];
-    if (act) {
-      const __nv_bfloat16* src = (kv == 0 ? k + t * k_stride : v + t * v_stride) + h * D + j * 8;
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    const __nv_bfloat16* src = (kv == 0 ? k + t * k_stride : v + t * v_stride) + h * D + j * 16;
+    const uint4 r0 = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    float x[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+    for (int i = 0; i < 8; ++i) {
+      x[2 * i] = __uint_as_float(wv[i] << 16);
+      x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
     }
-    // block amax over the 16 elements held by this thread and its partner
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    if (!act) continue;
-
-    const float g = __ldg(kv == 0 ? k_scale : v_scale);
-    const float s32 = __fdiv_rn(amax, __fmul_rn(6.0f, g));
-    const uint32_t sb = f32_to_e4m3(s32);
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const float g = kv == 0 ? gk : gv;
+    const uint32_t sb = e4m3_of_quotient(amax, __fmul_rn(6.0f, g));
     const float S = __fmul_rn(e4m3_to_f32(sb), g);
-    uint32_t packed = 0u;  // S == 0: every code 0
+    uint32_t c0 = 0u, c1 = 0u;  // S == 0: every code 0
     if (S >= 1.17549435e-38f) {
-      packed = e2m1_codes_div(x, S);
+      c0 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x), S);
+      c1 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x + 8), S);
     } else if (S > 0.0f) {  // subnormal effective scale: divide exactly
-      float q[8];
+      float q0[8], q1[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
-      packed = f32x8_to_e2m1x8(q);
+      for (int i = 0; i < 8; ++i) {
+        q0[i] = __fdiv_rn(x[i], S);
+        q1[i] = __fdiv_rn(x[8 + i], S);
+      }
+      c0 = f32x8_to_e2m1x8(q0);
+      c1 = f32x8_to_e2m1x8(q1);
     }
     uint8_t* dst =
         cache + (((blk * 2 + kv) * num_kv_heads + h) * (int64_t)block_size + off) * F;
-    *reinterpret_cast<uint32_t*>(dst + 4 * j) = packed;
-    if ((j & 1) == 0) dst[D / 2 + j / 2] = (uint8_t)sb;
+    if constexpr (F % 8 == 0) {  // rows 8-byte aligned
+      *reinterpret_cast<uint2*>(dst + 8 * j) = make_uint2(c0, c1);
+    } else {
+      reinterpret_cast<uint32_t*>(dst + 8 * j)[0] = c0;
+      reinterpret_cast<uint32_t*>(dst + 8 * j)[1] = c1;
+    }
+    dst[D / 2 + j] = (uint8_t)sb;
   }
 }
 
@@ -152,7 +168,9 @@ __global__ void __launch_bounds__(256) dequantize_paged_kernel(
 
 cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t stream) {
   const int bs_log2 = (a.block_size == 16) ? 4 : 5;  // validated: 16 or 32
-  const int block = 256;
+  // one thread per 16-element block of the token's 2 * num_kv_heads rows
+  const int rows_threads = 2 * a.num_kv_heads * (a.head_size / 16);
+  const int block = rows_threads <= 128 ? 128 : 256;
   if (a.num_tokens > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)a.num_tokens;
   const auto* k = static_cast<const __nv_bfloat16*>(a.k);
