@@ -229,9 +229,9 @@ class DecodeState:
         nk.quantize_append_paged(self.k_new, self.v_new, self.cache, self.slots, self.ks, self.vs,
                                  stream=stream)
 
-    def attend(self, nk, stream=None):
+    def attend(self, nk, stream=None, metadata_ready=False):
         nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
-                           self.ws, o_bf16=self.o16, stream=stream)
+                           self.ws, o_bf16=self.o16, stream=stream, metadata_ready=metadata_ready)
 
 
 def run_ours(args, rank, world, dist):
@@ -267,14 +267,16 @@ def run_ours(args, rank, world, dist):
         st.attend(nk, stream)
     stream.synchronize()
     # Per buffer copy: one CUDA graph for the whole step (append, then the
-    # attention kernel as its programmatic dependent) and one for the
-    # attention kernel alone (its own duration, timed back to back).
+    # attention kernel as its programmatic dependent; the block tables and
+    # lengths are step inputs the append does not write, so the attention
+    # kernel reads them while the append finishes) and one for the attention
+    # kernel alone (its own duration, timed back to back).
     g_step, g_att = [], []
     for st in states:
         ga = torch.cuda.CUDAGraph()
         with torch.cuda.graph(ga, stream=stream):
             st.append(nk, stream)
-            st.attend(nk, stream)
+            st.attend(nk, stream, metadata_ready=True)
         gb = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gb, stream=stream):
             st.attend(nk, stream)

@@ -157,6 +157,26 @@ NVFP4KV_API int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int
                           void* o_bf16, float* o_f32, void* workspace,
                           size_t workspace_bytes, nvfp4_stream_t stream);
 
+/* nvfp4_paged_attention with launch flags (no counterpart in the pages; a
+ * B200 launch option). The decode kernel is always launched as a programmatic
+ * dependent of the kernel before it on `stream`: its blocks may become
+ * resident while that kernel finishes, and by default they read nothing until
+ * it has completed. With NVFP4_ATTN_METADATA_READY the caller promises that
+ * block_table, seq_lens and qo_indptr are not written by that preceding
+ * kernel (they were made ready earlier, e.g. copied from the host before
+ * it); the kernel then loads them, builds its work split and fetches block
+ * ids before waiting, and reads q, the cache and the workspace only after.
+ * flags = 0 is nvfp4_paged_attention. Unknown bits: NVFP4_ERR_INVALID_ARG. */
+#define NVFP4_ATTN_METADATA_READY 0x1u
+NVFP4KV_API int nvfp4_paged_attention_ex(
+    const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
+    const uint8_t* cache, int64_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+    int32_t head_size, const int32_t* block_table, int32_t max_blocks_per_seq,
+    const int32_t* seq_lens, const int32_t* qo_indptr, int32_t num_seqs, int32_t max_q_len,
+    const float* kv_scales, float sm_scale, uint8_t* o_fp8, const float* o_scale,
+    void* o_bf16, float* o_f32, void* workspace, size_t workspace_bytes, uint32_t flags,
+    nvfp4_stream_t stream);
+
 /* Dequantize listed cache blocks to bf16 ("FlashInfer NVFP4 KV serving on
  * pre-SM100 GPUs", quick answer: the paged NVFP4 dequantize helper).
  *   block_ids       int32 [num_block_ids]: cache blocks to expand.

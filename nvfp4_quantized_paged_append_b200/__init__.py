@@ -26,6 +26,7 @@ NVFP4_ERR_WORKSPACE = -4
 DEV_BAD_SLOT = 0x1
 DEV_BAD_BLOCK = 0x2
 DEV_TIMEOUT = 0x4
+NVFP4_ATTN_METADATA_READY = 0x1
 
 
 class Nvfp4Error(RuntimeError):
@@ -66,6 +67,10 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_paged_attention.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P, i32, P, P,
                                         i32, i32, P, f32, P, P, P, P, P, sz, P]
     L.nvfp4_paged_attention.restype = ctypes.c_int
+    L.nvfp4_paged_attention_ex.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P, i32, P,
+                                           P, i32, i32, P, f32, P, P, P, P, P, sz,
+                                           ctypes.c_uint32, P]
+    L.nvfp4_paged_attention_ex.restype = ctypes.c_int
     L.nvfp4_paged_attention_noalloc.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P,
                                                 i32, P, P, i32, i32, P, f32, P, P, P, P, P]
     L.nvfp4_paged_attention_noalloc.restype = ctypes.c_int
@@ -161,8 +166,12 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                     qo_indptr: Optional[torch.Tensor] = None, max_q_len: int = 1,
                     sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
                     o_f32: Optional[torch.Tensor] = None,
-                    stream: Optional[torch.cuda.Stream] = None) -> None:
-    """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32)."""
+                    stream: Optional[torch.cuda.Stream] = None,
+                    metadata_ready: bool = False) -> None:
+    """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
+    metadata_ready: block_table, seq_lens and qo_indptr are not written by the
+    kernel launched just before on the stream, so the attention kernel may read
+    them while that kernel finishes (NVFP4_ATTN_METADATA_READY)."""
     nb, hkv, bs, d = _cache_dims(cache)
     tq, hq, dq = q.shape
     if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
@@ -176,11 +185,12 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                         ("o_f32", o_f32, torch.float32)):
         if o is not None and (o.dtype != dt or o.shape != (tq, hq, d) or not o.is_contiguous()):
             raise ValueError(f"{name} must be contiguous {dt} [Tq, Hq, D]")
-    st = lib().nvfp4_paged_attention(
+    st = lib().nvfp4_paged_attention_ex(
         _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
         _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream))
+        workspace.numel() * workspace.element_size(),
+        NVFP4_ATTN_METADATA_READY if metadata_ready else 0, _stream(stream))
     _check(st, "nvfp4_paged_attention")
 
 

@@ -95,6 +95,23 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
                           float sm_scale, uint8_t* o_fp8, const float* o_scale,
                           void* o_bf16, float* o_f32, void* workspace,
                           size_t workspace_bytes, nvfp4_stream_t stream) {
+  return nvfp4_paged_attention_ex(q, q_token_stride, num_q_tokens, num_q_heads, cache,
+                                  num_blocks, block_size, num_kv_heads, head_size, block_table,
+                                  max_blocks_per_seq, seq_lens, qo_indptr, num_seqs, max_q_len,
+                                  kv_scales, sm_scale, o_fp8, o_scale, o_bf16, o_f32, workspace,
+                                  workspace_bytes, 0u, stream);
+}
+
+int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                             int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                             int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                             const int32_t* block_table, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, const int32_t* qo_indptr,
+                             int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                             float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                             void* o_bf16, float* o_f32, void* workspace,
+                             size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
   if (num_q_tokens < 0 || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
       max_q_len < 0)
@@ -146,6 +163,7 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
   a.o_bf16 = o_bf16;
   a.o_f32 = o_f32;
   a.workspace = workspace;
+  a.flags = flags;
   cudaStream_t s = (cudaStream_t)stream;
   const int st = cuda_status(nvfp4kv::launch_decode_attention(a, s));
   if (st != NVFP4_OK) return st;

@@ -626,8 +626,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
 
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (when that kernel allows it): the block may be resident early, but reads
-  // nothing before that kernel has completed and its writes are visible.
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // nothing that kernel may write before it has completed and its writes are
+  // visible. With metadata_ready the batch metadata (sequence lengths, query
+  // ranges, block table) is known not to be among them and is read first.
+  const bool metadata_ready = (a.flags & kAttnMetadataReady) != 0;
+  if (!metadata_ready) grid_dependency_wait();
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   uint32_t* status = reinterpret_cast<uint32_t*>(a.workspace);
@@ -819,6 +822,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
     };
 
     batch_load(0);
+    if (metadata_ready) grid_dependency_wait();  // q, cache and workspace from here on
     {
       int b, h, ss;
       locate(s, b, h, ss);
@@ -1024,6 +1028,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   // ---- 3. cut segments. Every thread's partial writes are made visible
   // before the block's tickets; the ticket that completes a segment's count
   // of contributing warps makes this block its merger.
+  if (metadata_ready) grid_dependency_wait();  // (idle warps have not waited yet)
   __threadfence();
   __syncthreads();
   if (tid < 2 * nw) {

@@ -19,6 +19,13 @@ namespace nvfp4kv {
 constexpr uint32_t kDevBadSlot = 0x1u;
 constexpr uint32_t kDevBadBlock = 0x2u;
 constexpr uint32_t kDevTimeout = 0x4u;
+constexpr uint32_t kAttnMetadataReady = 0x1u;  // NVFP4_ATTN_METADATA_READY
+
+// Wait until the grids this one depends on (programmatic dependent launch)
+// have completed and their writes are visible; returns at once otherwise.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
 
 // ~ seconds of polling before a wait gives up (each try_wait suspends briefly).
 constexpr int kMaxWaitIters = 1 << 24;

@@ -56,6 +56,7 @@ struct AttentionArgs {
   void* o_bf16;   // may be null
   float* o_f32;   // may be null
   void* workspace;
+  uint32_t flags;  // NVFP4_ATTN_* launch flags (0: none)
 };
 
 // Decode split-KV: at most kDecodeWarps warps in the whole grid; every warp

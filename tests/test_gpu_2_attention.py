@@ -149,3 +149,45 @@ def test_output_scale_and_sm_scale_arguments():
     check_fp8(o8.cpu().numpy(), r8)
     assert ((r8.astype(np.int64) & 0x7F) == 0x7E).any()        # some outputs saturate at 448
     assert ((o8.cpu().numpy().astype(np.int64) & 0x7F) == 0x7E).any()
+
+
+def test_metadata_ready_after_writer_matches_default():
+    """The writer appends every sequence's last token, then attention runs as its
+    programmatic dependent with NVFP4_ATTN_METADATA_READY (block table and lengths
+    read before the writer finishes): outputs equal those of the default launch."""
+    w = wl.make_workload("qwen3_0p6b_decode")
+    scales = wl.global_scales(w, DEV)
+    k_scale, v_scale, o_scale = scales
+    B = w.num_seqs
+    hist = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, DEV)
+    ks = torch.tensor([k_scale], dtype=torch.float32, device=DEV)
+    vs = torch.tensor([v_scale], dtype=torch.float32, device=DEV)
+    k_new, v_new, slots = [], [], []
+    for b in range(B):
+        L = int(w.seq_lens[b])
+        k, v = wl.seq_kv(w, b, DEV)
+        nk.quantize_append_paged(k[:L - 1], v[:L - 1], hist,
+                                 torch.from_numpy(w.slots_for_seq(b, 0, L - 1)).to(DEV), ks, vs)
+        k_new.append(k[L - 1:])
+        v_new.append(v[L - 1:])
+        slots.append(w.slots_for_seq(b, L - 1)[:1])
+    k_new = torch.cat(k_new).contiguous()
+    v_new = torch.cat(v_new).contiguous()
+    slots = torch.from_numpy(np.concatenate(slots).astype(np.int64)).to(DEV)
+    q = wl.queries(w, DEV)
+    bt = torch.from_numpy(w.block_table).to(DEV)
+    sl = torch.from_numpy(w.seq_lens).to(DEV)
+    kvs = torch.tensor([k_scale, v_scale], dtype=torch.float32, device=DEV)
+    osc = torch.tensor([o_scale], dtype=torch.float32, device=DEV)
+    outs = []
+    for ready in (False, True):
+        cache = hist.clone()
+        ws = nk.alloc_workspace(B, w.num_q_heads, w.num_kv_heads, w.head_size, DEV)
+        o8 = torch.empty((B, w.num_q_heads, w.head_size), dtype=torch.uint8, device=DEV)
+        o32 = torch.empty((B, w.num_q_heads, w.head_size), dtype=torch.float32, device=DEV)
+        nk.quantize_append_paged(k_new, v_new, cache, slots, ks, vs)
+        nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, o_f32=o32, metadata_ready=ready)
+        torch.cuda.synchronize()
+        assert nk.workspace_status(ws) == 0
+        outs.append((o8, o32))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
