@@ -106,3 +106,31 @@ def test_dequant_validation(L):
     assert f(None, 10, 16, 8, 128, None, 4, None, None, None) == nk.NVFP4_ERR_INVALID_ARG
     assert f(None, 10, 16, 8, 128, None, 0, None, None, None) == nk.NVFP4_OK
     assert f(None, 10, 16, 8, 48, None, 4, None, None, None) == nk.NVFP4_ERR_UNSUPPORTED
+
+
+def _attn_ex(L, flags, **kw):
+    a = dict(q=None, qs=16 * 128, tq=4, hq=16, cache=None, nb=10, bs=16, hkv=8, D=128, bt=None,
+             mb=4, sl=None, qo=None, B=4, mq=1, kvs=None, sm=0.0, o8=None, osc=None, o16=None,
+             o32=None, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return L.nvfp4_paged_attention_ex(a["q"], a["qs"], a["tq"], a["hq"], a["cache"], a["nb"],
+                                      a["bs"], a["hkv"], a["D"], a["bt"], a["mb"], a["sl"], a["qo"],
+                                      a["B"], a["mq"], a["kvs"], a["sm"], a["o8"], a["osc"],
+                                      a["o16"], a["o32"], a["ws"], a["wsb"], flags, a["stream"])
+
+
+def test_attention_flags_and_output_alignment(L):
+    """Unknown launch flags are rejected; the known flag changes no validation.
+    Output pointers must allow the pair stores (fp8 2 B, bf16 4 B, fp32 8 B)."""
+    fake = ctypes.c_void_p(0x1000)
+    full = dict(q=fake, cache=fake, bt=fake, sl=fake, kvs=fake, o8=fake, osc=fake)
+    ready = nk.NVFP4_ATTN_METADATA_READY
+    assert _attn_ex(L, 0x2, **full) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, 0x80000000, B=0) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, ready, B=0) == nk.NVFP4_OK
+    assert _attn_ex(L, ready, **full) == nk.NVFP4_ERR_WORKSPACE      # same checks as flags = 0
+    assert _attn_ex(L, 0, **full) == _attn(L, **full)
+    ws = dict(ws=ctypes.c_void_p(0x100000), wsb=nk.workspace_size(4, 16, 8, 128))
+    assert _attn(L, **dict(full, o8=ctypes.c_void_p(0x1001)), **ws) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn(L, o16=ctypes.c_void_p(0x1002), **full, **ws) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn(L, o32=ctypes.c_void_p(0x1004), **full, **ws) == nk.NVFP4_ERR_INVALID_ARG
