@@ -3,11 +3,7 @@
 #include <math.h>
 
 #include "../../include/nvfp4kv.h"
-#include "nvfp4kv_launch.h"
-
-namespace nvfp4kv {
-int decode_warps(int head_size, int block_size, int num_seqs, int group);
-}
+#include "nvfp4kv_host.h"
 
 namespace {
 
@@ -17,13 +13,91 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 thread_local const char* g_last_error = "no error";
 
+}  // namespace
+
+namespace nvfp4kv {
+
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return NVFP4_OK;
   g_last_error = cudaGetErrorString(e);
   return NVFP4_ERR_CUDA;
 }
 
-}  // namespace
+AttentionArgs attention_args(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                             int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                             int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                             const int32_t* block_table, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, const int32_t* qo_indptr,
+                             int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                             float sm_scale, uint8_t* o_fp8, const float* o_scale, void* o_bf16,
+                             float* o_f32) {
+  AttentionArgs a{};
+  a.q = q;
+  a.q_token_stride = q_token_stride;
+  a.num_q_tokens = num_q_tokens;
+  a.num_q_heads = num_q_heads;
+  a.cache = cache;
+  a.num_blocks = num_blocks;
+  a.block_size = block_size;
+  a.num_kv_heads = num_kv_heads;
+  a.head_size = head_size;
+  a.block_table = block_table;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.seq_lens = seq_lens;
+  a.qo_indptr = qo_indptr;
+  a.num_seqs = num_seqs;
+  a.max_q_len = max_q_len;
+  a.kv_scales = kv_scales;
+  a.sm_scale = (sm_scale > 0.0f || head_size <= 0) ? sm_scale : 1.0f / sqrtf((float)head_size);
+  a.o_fp8 = o_fp8;
+  a.o_scale = o_scale;
+  a.o_bf16 = o_bf16;
+  a.o_f32 = o_f32;
+  return a;
+}
+
+int check_attention(const AttentionArgs& a, bool* nothing_to_do) {
+  *nothing_to_do = false;
+  if (a.num_q_tokens < 0 || a.num_seqs < 0 || a.num_q_heads <= 0 || a.num_kv_heads <= 0 ||
+      a.head_size <= 0 || a.block_size <= 0 || a.num_blocks <= 0 || a.max_blocks_per_seq <= 0 ||
+      a.max_q_len < 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (a.head_size % 16 != 0 || a.num_q_heads % a.num_kv_heads != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!head_size_ok(a.head_size) || !block_size_ok(a.block_size)) return NVFP4_ERR_UNSUPPORTED;
+  const int G = a.num_q_heads / a.num_kv_heads;
+  if (G > 8) return NVFP4_ERR_UNSUPPORTED;
+  if (!a.qo_indptr && a.num_q_tokens < a.num_seqs) return NVFP4_ERR_INVALID_ARG;
+  if (!a.qo_indptr && a.max_q_len > 1) return NVFP4_ERR_INVALID_ARG;
+  if (a.num_seqs == 0 || a.num_q_tokens == 0) {
+    *nothing_to_do = true;
+    return NVFP4_OK;
+  }
+  if (!a.q || !a.cache || !a.block_table || !a.seq_lens || !a.kv_scales || !a.o_fp8 ||
+      !a.o_scale)
+    return NVFP4_ERR_INVALID_ARG;
+  if (a.q_token_stride < (int64_t)a.num_q_heads * a.head_size || a.q_token_stride % 8 != 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(a.q, 16) || !aligned(a.cache, 16) || !aligned(a.o_fp8, 2) ||
+      (a.o_bf16 && !aligned(a.o_bf16, 4)) || (a.o_f32 && !aligned(a.o_f32, 8)))
+    return NVFP4_ERR_INVALID_ARG;
+  // flattened page indices and cache page rows are int32 on the device
+  if ((int64_t)a.num_seqs * a.max_blocks_per_seq * a.num_kv_heads >= (int64_t)1 << 30 ||
+      a.num_blocks * 2 * a.num_kv_heads >= (int64_t)1 << 31)
+    return NVFP4_ERR_UNSUPPORTED;
+  if (decode_warps(a.head_size, a.block_size, a.num_seqs, G) < 1) return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+int launch_attention(const AttentionArgs& a, cudaStream_t s) {
+  const int st = cuda_status(launch_decode_attention(a, s));
+  if (st != NVFP4_OK) return st;
+  if (a.qo_indptr && a.max_q_len > 1) return cuda_status(launch_prefill_attention(a, s));
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4kv
+
+using nvfp4kv::cuda_status;
 
 extern "C" {
 
@@ -112,63 +186,19 @@ int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_
                              void* o_bf16, float* o_f32, void* workspace,
                              size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
   if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
-  if (num_q_tokens < 0 || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-      head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
-      max_q_len < 0)
-    return NVFP4_ERR_INVALID_ARG;
-  if (head_size % 16 != 0 || num_q_heads % num_kv_heads != 0) return NVFP4_ERR_INVALID_ARG;
-  if (!head_size_ok(head_size) || !block_size_ok(block_size)) return NVFP4_ERR_UNSUPPORTED;
-  const int G = num_q_heads / num_kv_heads;
-  if (G > 8) return NVFP4_ERR_UNSUPPORTED;
-  if (!qo_indptr && num_q_tokens < num_seqs) return NVFP4_ERR_INVALID_ARG;
-  if (!qo_indptr && max_q_len > 1) return NVFP4_ERR_INVALID_ARG;
-  if (num_seqs == 0 || num_q_tokens == 0) return NVFP4_OK;
-  if (!q || !cache || !block_table || !seq_lens || !kv_scales || !o_fp8 || !o_scale)
-    return NVFP4_ERR_INVALID_ARG;
-  if (q_token_stride < (int64_t)num_q_heads * head_size || q_token_stride % 8 != 0)
-    return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(cache, 16) || !aligned(o_fp8, 2) ||
-      (o_bf16 && !aligned(o_bf16, 4)) || (o_f32 && !aligned(o_f32, 8)))
-    return NVFP4_ERR_INVALID_ARG;
-  // flattened page indices and cache page rows are int32 on the device
-  if ((int64_t)num_seqs * max_blocks_per_seq * num_kv_heads >= (int64_t)1 << 30 ||
-      num_blocks * 2 * num_kv_heads >= (int64_t)1 << 31)
-    return NVFP4_ERR_UNSUPPORTED;
-  if (nvfp4kv::decode_warps(head_size, block_size, num_seqs, num_q_heads / num_kv_heads) < 1)
-    return NVFP4_ERR_UNSUPPORTED;
+  nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
+      q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
+      head_size, block_table, max_blocks_per_seq, seq_lens, qo_indptr, num_seqs, max_q_len,
+      kv_scales, sm_scale, o_fp8, o_scale, o_bf16, o_f32);
+  bool nothing_to_do = false;
+  const int st = nvfp4kv::check_attention(a, &nothing_to_do);
+  if (st != NVFP4_OK || nothing_to_do) return st;
   const size_t need = nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
                                                            head_size);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return NVFP4_ERR_WORKSPACE;
-
-  nvfp4kv::AttentionArgs a{};
-  a.q = q;
-  a.q_token_stride = q_token_stride;
-  a.num_q_tokens = num_q_tokens;
-  a.num_q_heads = num_q_heads;
-  a.cache = cache;
-  a.num_blocks = num_blocks;
-  a.block_size = block_size;
-  a.num_kv_heads = num_kv_heads;
-  a.head_size = head_size;
-  a.block_table = block_table;
-  a.max_blocks_per_seq = max_blocks_per_seq;
-  a.seq_lens = seq_lens;
-  a.qo_indptr = qo_indptr;
-  a.num_seqs = num_seqs;
-  a.max_q_len = max_q_len;
-  a.kv_scales = kv_scales;
-  a.sm_scale = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)head_size);
-  a.o_fp8 = o_fp8;
-  a.o_scale = o_scale;
-  a.o_bf16 = o_bf16;
-  a.o_f32 = o_f32;
   a.workspace = workspace;
   a.flags = flags;
-  cudaStream_t s = (cudaStream_t)stream;
-  const int st = cuda_status(nvfp4kv::launch_decode_attention(a, s));
-  if (st != NVFP4_OK) return st;
-  if (qo_indptr && max_q_len > 1) return cuda_status(nvfp4kv::launch_prefill_attention(a, s));
-  return NVFP4_OK;
+  return nvfp4kv::launch_attention(a, (cudaStream_t)stream);
 }
 
 int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks, int32_t block_size,
