@@ -74,6 +74,8 @@ EDGE = [
     (128, 16, 16, 8, [40, 300, 16], [40, 77, 2]),           # q_len == L (no cache) / ragged
     (256, 32, 16, 2, [200, 64], [130, 64]),                 # G = 8, bs 32 prefill
     (128, 16, 8, 2, [5], [9]),                              # q_len > L: early rows see nothing
+    (128, 16, 12, 4, [100, 700, 2500], None),               # G = 3: odd group, lo columns cross lanes
+    (64, 16, 12, 2, [90, 1300], None),                      # G = 6: separate lo fragments
 ]
 
 
