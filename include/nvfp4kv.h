@@ -162,10 +162,11 @@ NVFP4KV_API int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int
  * dependent of the kernel before it on `stream`: its blocks may become
  * resident while that kernel finishes, and by default they read nothing until
  * it has completed. With NVFP4_ATTN_METADATA_READY the caller promises that
- * block_table, seq_lens and qo_indptr are not written by that preceding
- * kernel (they were made ready earlier, e.g. copied from the host before
- * it); the kernel then loads them, builds its work split and fetches block
- * ids before waiting, and reads q, the cache and the workspace only after.
+ * the preceding kernel writes none of block_table, seq_lens, qo_indptr,
+ * kv_scales, o_scale and the workspace (they were made ready earlier, e.g.
+ * copied from the host before it); the kernel then reads them, builds its
+ * work split, fetches block ids (setting NVFP4_DEV_BAD_BLOCK in the status
+ * word for bad ones) before waiting, and reads q and the cache only after.
  * flags = 0 is nvfp4_paged_attention. Unknown bits: NVFP4_ERR_INVALID_ARG. */
 #define NVFP4_ATTN_METADATA_READY 0x1u
 NVFP4KV_API int nvfp4_paged_attention_ex(

@@ -169,9 +169,10 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                     stream: Optional[torch.cuda.Stream] = None,
                     metadata_ready: bool = False) -> None:
     """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
-    metadata_ready: block_table, seq_lens and qo_indptr are not written by the
-    kernel launched just before on the stream, so the attention kernel may read
-    them while that kernel finishes (NVFP4_ATTN_METADATA_READY)."""
+    metadata_ready: the kernel launched just before on the stream writes none of
+    block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
+    attention kernel may read them while that kernel finishes
+    (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it)."""
     nb, hkv, bs, d = _cache_dims(cache)
     tq, hq, dq = q.shape
     if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
