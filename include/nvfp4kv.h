@@ -205,7 +205,7 @@ NVFP4KV_API int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
  * (nvfp4_paged_attention_workspace_size) exceeds it return
  * NVFP4_ERR_WORKSPACE. The first call on a device looks up the array's
  * device address on that device (make that first call before any stream
- * capture). Each call clears the array's status word and completion tickets
+ * capture). Each call clears the array's status word and arrival counters
  * on `stream` first; all calls share the one array, so calls that may
  * overlap on the GPU (unordered streams) race and must not be made. The
  * call never calls cudaMalloc, cudaFree or any allocating routine. */

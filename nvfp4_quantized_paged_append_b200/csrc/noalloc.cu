@@ -1,7 +1,7 @@
 // Paged attention without a caller-provided workspace.
 //
 // nvfp4_paged_attention needs scratch memory for its split-KV partial
-// results, completion tickets and status word, and takes it from the caller.
+// results, arrival counters and status word, and takes it from the caller.
 // Some callers have no way to supply it: code handed only its input and
 // output buffers by a host framework (a plugin or callback interface with no
 // workspace hook), or code running while the device memory is owned by
@@ -16,7 +16,7 @@
 // (with that device current) and caches it; do that first call outside any
 // stream capture. All calls on a device share the array and the array keeps
 // whatever the previous call left in it, so each call clears the part that
-// must start at zero (status word and completion tickets) on its stream
+// must start at zero (status word and arrival counters) on its stream
 // before the kernels run. Calls that overlap on the GPU (different streams,
 // no ordering between them) race on the array and must not be issued.
 #include <mutex>

@@ -92,7 +92,7 @@ def test_edge_cases(D, bs, hq, hkv, lens, qlens):
 
 
 def test_repeat_calls_identical_and_workspace_reusable():
-    """Split-KV tickets reset themselves: a second call on the same workspace
+    """Split-KV arrival counters reset themselves: a second call on the same workspace
     gives bit-identical outputs."""
     w = wl.make_workload("qwen3_0p6b_decode")
     scales = wl.global_scales(w, DEV)
