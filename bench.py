@@ -91,12 +91,21 @@ def barrier(dist):
 
 
 def max_over_ranks(x, dist):
+    """The largest x over all ranks (the job's time is its slowest rank's)."""
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(ms_local, steps, bytes_per_step, dist, world):
+    """(ms per step, whole-job GB/s): every rank processes bytes_per_step per
+    step (replicas, weak scaling) and the job takes its slowest rank's time."""
+    ms_step = max_over_ranks(ms_local, dist) / steps
+    return ms_step, world * bytes_per_step / (ms_step * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------------ clocks
@@ -315,8 +324,7 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     barrier(dist)
     ms_local = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms_local, dist)
-    ms_step = ms / args.steps
+    ms_step, value = job_throughput(ms_local, args.steps, kv_bytes, dist, world)
     clocks.stop()
     # the attention kernel's own average duration: the same number of
     # attention-only launches back to back on the launching stream
@@ -389,7 +397,7 @@ def run_ours(args, rank, world, dist):
     traffic = profiled_traffic("decode_attention_kernel<128,16>", WORKLOAD)
     result = {
         "metric": METRIC,
-        "value": round(world * kv_bytes / (ms_step * 1e-3) / 1e9, 2),
+        "value": round(value, 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
