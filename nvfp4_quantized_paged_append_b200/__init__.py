@@ -160,19 +160,9 @@ def workspace_status(workspace: torch.Tensor) -> int:
     return int(workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
 
 
-def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
-                    seq_lens: torch.Tensor, kv_scales: torch.Tensor, o_fp8: torch.Tensor,
-                    o_scale: torch.Tensor, workspace: torch.Tensor,
-                    qo_indptr: Optional[torch.Tensor] = None, max_q_len: int = 1,
-                    sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
-                    o_f32: Optional[torch.Tensor] = None,
-                    stream: Optional[torch.cuda.Stream] = None,
-                    metadata_ready: bool = False) -> None:
-    """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
-    metadata_ready: the kernel launched just before on the stream writes none of
-    block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
-    attention kernel may read them while that kernel finishes
-    (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it)."""
+def _attention_dims(q, cache, block_table, seq_lens, qo_indptr, o_fp8, o_bf16, o_f32):
+    """Shape and dtype checks shared by the attention calls; returns
+    (num_blocks, Hkv, block_size, D, Tq, Hq, num_seqs, max_blocks_per_seq)."""
     nb, hkv, bs, d = _cache_dims(cache)
     tq, hq, dq = q.shape
     if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
@@ -186,6 +176,24 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                         ("o_f32", o_f32, torch.float32)):
         if o is not None and (o.dtype != dt or o.shape != (tq, hq, d) or not o.is_contiguous()):
             raise ValueError(f"{name} must be contiguous {dt} [Tq, Hq, D]")
+    return nb, hkv, bs, d, tq, hq, B, mb
+
+
+def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
+                    seq_lens: torch.Tensor, kv_scales: torch.Tensor, o_fp8: torch.Tensor,
+                    o_scale: torch.Tensor, workspace: torch.Tensor,
+                    qo_indptr: Optional[torch.Tensor] = None, max_q_len: int = 1,
+                    sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
+                    o_f32: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None,
+                    metadata_ready: bool = False) -> None:
+    """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
+    metadata_ready: the kernel launched just before on the stream writes none of
+    block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
+    attention kernel may read them while that kernel finishes
+    (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it)."""
+    nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, qo_indptr,
+                                                    o_fp8, o_bf16, o_f32)
     st = lib().nvfp4_paged_attention_ex(
         _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
@@ -206,11 +214,8 @@ def paged_attention_noalloc(q: torch.Tensor, cache: torch.Tensor, block_table: t
     library uses its own fixed scratch array (see nvfp4_paged_attention_noalloc
     in include/nvfp4kv.h: one array per GPU, shared by all calls, so calls must
     not overlap on the GPU; sizes beyond it raise)."""
-    nb, hkv, bs, d = _cache_dims(cache)
-    tq, hq, dq = q.shape
-    if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
-        raise ValueError("q must be bf16 [Tq, Hq, D] with contiguous heads")
-    B, mb = block_table.shape
+    nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, qo_indptr,
+                                                    o_fp8, o_bf16, o_f32)
     st = lib().nvfp4_paged_attention_noalloc(
         _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),

@@ -134,3 +134,34 @@ def test_attention_flags_and_output_alignment(L):
     assert _attn(L, **dict(full, o8=ctypes.c_void_p(0x1001)), **ws) == nk.NVFP4_ERR_INVALID_ARG
     assert _attn(L, o16=ctypes.c_void_p(0x1002), **full, **ws) == nk.NVFP4_ERR_INVALID_ARG
     assert _attn(L, o32=ctypes.c_void_p(0x1004), **full, **ws) == nk.NVFP4_ERR_INVALID_ARG
+
+
+def test_binding_rejects_bad_attention_tensors(L):
+    """The Python binding checks shapes and dtypes (both attention calls) before
+    any pointer reaches the library."""
+    import torch
+    cache = torch.zeros((4, 2, 2, 16, 72), dtype=torch.uint8)
+    q = torch.zeros((2, 4, 128), dtype=torch.bfloat16)
+    bt = torch.zeros((2, 3), dtype=torch.int32)
+    sl = torch.ones(2, dtype=torch.int32)
+    kvs = torch.ones(2)
+    o8 = torch.zeros((2, 4, 128), dtype=torch.uint8)
+    osc = torch.ones(1)
+    ws = torch.zeros(1024, dtype=torch.uint8)
+    for call in (lambda **kw: nk.paged_attention(workspace=ws, **kw),
+                 lambda **kw: nk.paged_attention_noalloc(**kw)):
+        def run(**over):
+            args = dict(q=q, cache=cache, block_table=bt, seq_lens=sl, kv_scales=kvs, o_fp8=o8,
+                        o_scale=osc)
+            args.update(over)
+            return call(**args)
+        with pytest.raises(ValueError):
+            run(q=q.float())                                   # q dtype
+        with pytest.raises(ValueError):
+            run(block_table=bt.long())                         # block table dtype
+        with pytest.raises(ValueError):
+            run(seq_lens=sl.long())                            # lengths dtype
+        with pytest.raises(ValueError):
+            run(o_fp8=torch.zeros((2, 4, 64), dtype=torch.uint8))  # output shape
+        with pytest.raises(ValueError):
+            run(cache=torch.zeros((4, 2, 2, 16, 70), dtype=torch.uint8))  # not a full_dim
