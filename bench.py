@@ -58,6 +58,10 @@ def parse():
                    help="kernel-only mode for profilers: set up, then launch the chosen "
                         "kernel --steps times (no timing, no JSON)")
     p.add_argument("--workload", default=WORKLOAD, help="workload for --profile attention")
+    p.add_argument("--time-workloads", default=None,
+                   help="comma-separated workload names (e.g. long_decode,mixed_prefill_decode):"
+                        " time one attention call per workload, L2 flushed before each, and"
+                        " print one JSON line each instead of the benchmark line")
     return p.parse_args()
 
 
@@ -530,6 +534,64 @@ def run_reference(args, rank, world):
     }
 
 
+def run_workload_times(args):
+    """One attention call per named workload (its own cache, filled by the
+    writer), after a 256 MiB write that evicts L2; median of 10 event-timed
+    calls after 2 warm-ups. KV GB/s counts the K+V rows the call must read;
+    for multi-token query ranges the causal prefill FLOPs are reported too
+    (the call's time covers both the decode and the prefill kernel)."""
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for name in args.time_workloads.split(","):
+        w = wl.make_workload(name.strip())
+        scales = wl.global_scales(w, dev)
+        cache = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+        ks = torch.tensor([scales[0]], device=dev)
+        vs = torch.tensor([scales[1]], device=dev)
+        for b in range(w.num_seqs):
+            k, v = wl.seq_kv(w, b, dev)
+            nk.quantize_append_paged(k, v, cache, torch.from_numpy(w.slots_for_seq(b)).to(dev),
+                                     ks, vs)
+        q = wl.queries(w, dev)
+        o8 = torch.empty((w.num_q_tokens, w.num_q_heads, w.head_size), dtype=torch.uint8,
+                         device=dev)
+        ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, dev)
+        bt = torch.from_numpy(w.block_table).to(dev)
+        sl = torch.from_numpy(w.seq_lens).to(dev)
+        qo = None if w.is_decode else torch.from_numpy(w.qo_indptr).to(dev)
+        kvs = torch.tensor([scales[0], scales[1]], device=dev)
+        osc = torch.tensor([scales[2]], device=dev)
+        times = []
+        for i in range(12):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, qo_indptr=qo,
+                               max_q_len=w.max_q_len)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1) * 1e3)
+        us = statistics.median(times)
+        gbs = w.kv_bytes() / (us * 1e-6) / 1e9
+        line = {"workload": name.strip(), "call_us": round(us, 2), "kv_bytes": w.kv_bytes(),
+                "kv_gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+                "frac_of_8TBps": round(gbs / 8000.0, 4), "peak_kind": peak_kind,
+                "timing": "median of 10 single calls, L2 evicted before each"}
+        flops = w.prefill_flops()
+        if flops:
+            line["prefill_flops"] = flops
+            line["prefill_tflops_over_call"] = round(flops / (us * 1e-6) / 1e12, 1)
+        print(json.dumps(line), flush=True)
+        del cache, ws
+        torch.cuda.empty_cache()
+
+
 def run_profile(args):
     """Set up one workload and launch one kernel --steps times (for ncu)."""
     import torch
@@ -577,6 +639,9 @@ def main():
     args = parse()
     if args.profile:
         run_profile(args)
+        return
+    if args.time_workloads:
+        run_workload_times(args)
         return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

@@ -103,6 +103,18 @@ class PagedWorkload:
         """NVFP4 K+V row bytes the attention must read (no block padding)."""
         return int(self.seq_lens.astype(np.int64).sum()) * self.num_kv_heads * 2 * self.full_dim
 
+    def prefill_flops(self) -> int:
+        """Causal QK^T + PV FLOPs of the multi-token query ranges: 4 * D per
+        (query row, visible key, query head)."""
+        total = 0
+        for b in range(self.num_seqs):
+            ql, L = int(self.q_lens[b]), int(self.seq_lens[b])
+            if ql <= 1:
+                continue
+            p = L - ql + np.arange(ql, dtype=np.int64)   # absolute position of each row
+            total += int(np.clip(p + 1, 0, None).sum())
+        return total * self.num_q_heads * 4 * self.head_size
+
     def slots_for_seq(self, b: int, start: int = 0, stop: Optional[int] = None) -> np.ndarray:
         """Cache slots of tokens start..stop-1 of sequence b (int64)."""
         stop = int(self.seq_lens[b]) if stop is None else stop
