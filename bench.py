@@ -19,8 +19,12 @@ ranks (each rank runs its own replica: the path has no exchange step).
 
 Also reported: roofline of the attention kernel (its own CUDA-event time per
 launch), the quantize-append sweep (8192 tokens into a 65536 x 16 cache) in
-Mtok/s, the end-to-end number through host buffers, the CPU oracle baseline
-and SM clocks sampled during the timed region.
+Mtok/s, the long-context decode batch (64 x 32768 keys, 2.4 GB of KV) in KV
+GB/s, the mixed chunked-prefill batch (8 x 2048 causal queries over 10240
+keys plus 56 decode sequences, head_size 256, GQA 8) as the whole call and as
+its prefill (TFLOP/s against the sustained bf16 tensor peak) and decode
+sub-batches, the end-to-end number through host buffers, the CPU oracle
+baseline and SM clocks sampled during each timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -45,6 +49,8 @@ METRIC = "NVFP4 paged decode attn KV GB/s (% of HBM peak); append Mtok/s"
 WORKLOAD = "qwen3_0p6b_decode"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 
 def parse():
@@ -72,6 +78,17 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peaks():
+    """(burst, sustained) dense bf16 TFLOP/s and their kind."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            "measured"
+    return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
 # ------------------------------------------------------------------ distributed
@@ -153,10 +170,14 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, region=0):
+        """Clocks over the region between marks 2*region and 2*region + 1."""
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, time.time())
+        if len(self.marks) >= 2 * region + 2:
+            t0, t1 = self.marks[2 * region], self.marks[2 * region + 1]
+        else:
+            t0, t1 = 0, time.time()
         rows = [s for t, s in self.samples if t0 - 0.15 <= t <= t1 + 0.15] or \
                [s for _, s in self.samples[-5:]]
         mhz, mx, reasons = [], None, set()
@@ -209,16 +230,16 @@ def profiled_traffic(kernel, workload):
 
 
 class DecodeState:
-    """One independent copy of the step's device state."""
+    """One independent copy of the step's device state. The step's host inputs
+    (q, new k/v, slots, seq_lens, block table) live in one device staging
+    buffer, so the end-to-end loop moves them with a single host-to-device
+    copy per step."""
 
     def __init__(self, w, scales, hist_cache, device):
         import torch
         import nvfp4_quantized_paged_append_b200 as nk
         from nvfp4_quantized_paged_append_b200 import workloads as wl
         self.cache = hist_cache.clone()
-        self.bt = torch.from_numpy(w.block_table).to(device)
-        self.sl = torch.from_numpy(w.seq_lens).to(device)
-        self.q = wl.queries(w, device)
         B, H, D = w.num_seqs, w.num_kv_heads, w.head_size
         # the new token of each sequence = its last position
         ks, vs = [], []
@@ -226,10 +247,21 @@ class DecodeState:
             k, v = wl.seq_kv(w, b, device, start=int(w.seq_lens[b]) - 1)
             ks.append(k)
             vs.append(v)
-        self.k_new = torch.cat(ks).contiguous()
-        self.v_new = torch.cat(vs).contiguous()
-        self.slots = torch.from_numpy(np.array(
-            [w.slots_for_seq(b, int(w.seq_lens[b]) - 1)[0] for b in range(B)], np.int64)).to(device)
+        slots = torch.from_numpy(np.array(
+            [w.slots_for_seq(b, int(w.seq_lens[b]) - 1)[0] for b in range(B)], np.int64))
+        parts = [("q", wl.queries(w, device)), ("k_new", torch.cat(ks)), ("v_new", torch.cat(vs)),
+                 ("slots", slots), ("sl", torch.from_numpy(w.seq_lens)),
+                 ("bt", torch.from_numpy(w.block_table))]
+        offs, total = [], 0
+        for _, t in parts:
+            offs.append(total)
+            total += -(-t.numel() * t.element_size() // 256) * 256
+        self.stage = torch.zeros(total, dtype=torch.uint8, device=device)
+        for (name, t), off in zip(parts, offs):
+            n = t.numel() * t.element_size()
+            view = self.stage[off:off + n].view(t.dtype).view(t.shape)
+            view.copy_(t)
+            setattr(self, name, view)
         self.kvs = torch.tensor([scales[0], scales[1]], dtype=torch.float32, device=device)
         self.ks = self.kvs[0:1]
         self.vs = self.kvs[1:2]
@@ -245,6 +277,140 @@ class DecodeState:
     def attend(self, nk, stream=None, metadata_ready=False):
         nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
                            self.ws, o_bf16=self.o16, stream=stream, metadata_ready=metadata_ready)
+
+
+def build_cache(w, scales, dev):
+    """The workload's whole cache, written by the library's writer."""
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    cache = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+    ks = torch.tensor([scales[0]], dtype=torch.float32, device=dev)
+    vs = torch.tensor([scales[1]], dtype=torch.float32, device=dev)
+    for b in range(w.num_seqs):
+        k, v = wl.seq_kv(w, b, dev)
+        nk.quantize_append_paged(k, v, cache, torch.from_numpy(w.slots_for_seq(b)).to(dev), ks, vs)
+    return cache
+
+
+class AttentionCall:
+    """Device inputs/outputs of one attention call over a workload (or a
+    sub-batch of one, sharing its cache)."""
+
+    def __init__(self, w, cache, q, scales, dev):
+        import torch
+        import nvfp4_quantized_paged_append_b200 as nk
+        self.nk, self.w, self.cache, self.q = nk, w, cache, q
+        self.bt = torch.from_numpy(w.block_table).to(dev)
+        self.sl = torch.from_numpy(w.seq_lens).to(dev)
+        self.qo = None if w.is_decode else torch.from_numpy(w.qo_indptr).to(dev)
+        self.kvs = torch.tensor([scales[0], scales[1]], dtype=torch.float32, device=dev)
+        self.osc = torch.tensor([scales[2]], dtype=torch.float32, device=dev)
+        shape = (w.num_q_tokens, w.num_q_heads, w.head_size)
+        self.o8 = torch.empty(shape, dtype=torch.uint8, device=dev)
+        self.o16 = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        self.ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, dev)
+
+    def __call__(self, stream):
+        self.nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
+                                self.ws, qo_indptr=self.qo, max_q_len=self.w.max_q_len,
+                                o_bf16=self.o16, stream=stream)
+
+
+def time_calls(fn, n, stream, warm=3):
+    """Mean milliseconds per call of n back-to-back calls on `stream`
+    (CUDA events on that stream), after `warm` untimed calls."""
+    import torch
+    for _ in range(warm):
+        fn(stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        fn(stream)
+    e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def long_decode_record(stream, clocks, region, n_calls=20):
+    """Long-context decode (64 sequences x 32768 keys, 32 q / 8 kv heads,
+    head_size 128, block_size 32; 2.4 GB of NVFP4 KV, far above L2): n
+    back-to-back attention calls."""
+    import torch
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.make_workload("long_decode")
+    scales = wl.global_scales(w, dev)
+    cache = build_cache(w, scales, dev)
+    call = AttentionCall(w, cache, wl.queries(w, dev), scales, dev)
+    time_calls(call, 3, stream, warm=2)
+    clocks.mark()
+    ms = time_calls(call, n_calls, stream)
+    clocks.mark()
+    peak, kind = peaks()
+    gbs = w.kv_bytes() / (ms * 1e-3) / 1e9
+    rec = {"workload": "long_decode", "kernel": "decode_attention_kernel<128,32>",
+           "calls": n_calls, "kernel_ms": round(ms, 5), "kv_bytes": w.kv_bytes(),
+           "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "peak": peak,
+           "peak_kind": f"{kind} HBM copy", "frac_of_8TBps": round(gbs / 8000.0, 4),
+           "l2": "2.4 GB of KV per call (> 19x L2)", "clocks": clocks.summary(region)}
+    del cache, call
+    torch.cuda.empty_cache()
+    return rec
+
+
+def mixed_record(stream, clocks, region, n_prefill=5, n_decode=20):
+    """Mixed chunked prefill + decode (64 q / 8 kv heads, head_size 256,
+    block_size 16; 8 sequences prefilling 2048 causal queries over 8192 cached
+    keys, 56 decode sequences of 1024-16384 keys). Timed as the whole mixed
+    call, and as its prefill and decode sub-batches alone (same cache)."""
+    import torch
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.make_workload("mixed_prefill_decode")
+    scales = wl.global_scales(w, dev)
+    cache = build_cache(w, scales, dev)
+    q = wl.queries(w, dev)
+    pre_seqs = [b for b in range(w.num_seqs) if w.q_lens[b] > 1]
+    dec_seqs = [b for b in range(w.num_seqs) if w.q_lens[b] == 1]
+    wp, tp = w.subset(pre_seqs)
+    wd, td = w.subset(dec_seqs)
+    full = AttentionCall(w, cache, q, scales, dev)
+    pre = AttentionCall(wp, cache, q[torch.from_numpy(tp).to(dev)].contiguous(), scales, dev)
+    dec = AttentionCall(wd, cache, q[torch.from_numpy(td).to(dev)].contiguous(), scales, dev)
+    time_calls(full, 1, stream, warm=1)
+    clocks.mark()
+    ms_full = time_calls(full, n_prefill, stream)
+    ms_pre = time_calls(pre, n_prefill, stream)
+    ms_dec = time_calls(dec, n_decode, stream)
+    clocks.mark()
+    burst, sustained, tkind = tensor_peaks()
+    peak, kind = peaks()
+    flops = w.prefill_flops()
+    tf = flops / (ms_pre * 1e-3) / 1e12
+    dgbs = wd.kv_bytes() / (ms_dec * 1e-3) / 1e9
+    rec = {"workload": "mixed_prefill_decode",
+           "call_ms": round(ms_full, 4),
+           "call_tflops_prefill_over_call": round(flops / (ms_full * 1e-3) / 1e12, 1),
+           "prefill": {"kernel": "prefill attention (8 seqs x 2048 causal queries over 10240 keys)",
+                       "ms": round(ms_pre, 4), "flops": flops, "tflops": round(tf, 1),
+                       "peak": sustained, "unit": "TFLOP/s",
+                       "peak_kind": f"{tkind} dense bf16, sustained (seconds-long loop)",
+                       "frac": round(tf / sustained, 4),
+                       "frac_of_burst": round(tf / burst, 4),
+                       "prefill_kv_bytes": wp.kv_bytes()},
+           "decode": {"kernel": "decode_attention_kernel<256,16>", "ms": round(ms_dec, 5),
+                      "kv_bytes": wd.kv_bytes(), "gbs": round(dgbs, 1),
+                      "frac": round(dgbs / peak, 4), "peak": peak,
+                      "peak_kind": f"{kind} HBM copy"},
+           "timing": f"back-to-back calls: {n_prefill} mixed, {n_prefill} prefill-only, "
+                     f"{n_decode} decode-only (CUDA events on the launching stream)",
+           "clocks": clocks.summary(region)}
+    del cache, full, pre, dec
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args, rank, world, dist):
@@ -329,7 +495,6 @@ def run_ours(args, rank, world, dist):
     barrier(dist)
     ms_local = e0.elapsed_time(e1)
     ms_step, value = job_throughput(ms_local, args.steps, kv_bytes, dist, world)
-    clocks.stop()
     # the attention kernel's own average duration: the same number of
     # attention-only launches back to back on the launching stream
     run_attention(max(3, args.warmup))
@@ -354,47 +519,50 @@ def run_ours(args, rank, world, dist):
     kas = [ka.clone() for _ in range(acopies)]
     vas = [va.clone() for _ in range(acopies)]
     nrep = 400
-    if True:
-        for i in range(20):
-            nk.quantize_append_paged(kas[i % acopies], vas[i % acopies], acache, slots, ksa, vsa,
-                                     stream=stream)
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for i in range(nrep):
-            nk.quantize_append_paged(kas[i % acopies], vas[i % acopies], acache, slots, ksa, vsa,
-                                     stream=stream)
-        a1.record(stream)
-    stream.synchronize()
-    app_ms = a0.elapsed_time(a1) / nrep
-    app_bytes = app.algorithmic_bytes()
+    it = [0]
 
-    # ---- end to end through host buffers (pinned), every step: H2D of q, new k/v,
-    # slots, seq_lens, block table; D2H of the bf16 output
-    st = states[0]
-    host_in = {name: getattr(st, name).cpu().pin_memory()
-               for name in ("q", "k_new", "v_new", "slots", "sl", "bt")}
-    host_out = torch.empty_like(st.o16, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    def append_once(s):
+        i = it[0]
+        it[0] += 1
+        nk.quantize_append_paged(kas[i % acopies], vas[i % acopies], acache, slots, ksa, vsa,
+                                 stream=s)
+
+    app_ms = time_calls(append_once, nrep, stream, warm=20)
+    app_bytes = app.algorithmic_bytes()
+    del kas, vas, acache
+    torch.cuda.empty_cache()
+
+    # ---- end to end through host buffers (pinned), every step: one H2D copy
+    # of the packed step inputs (q, new k/v, slots, seq_lens, block table),
+    # the append and attention calls, and a D2H copy of the bf16 output
+    host_stage = states[0].stage.cpu().pin_memory()
+    host_out = torch.empty_like(states[0].o16, device="cpu").pin_memory()
+    h2d = host_stage.numel()
     d2h = host_out.numel() * host_out.element_size()
     e2e_steps = max(50, min(500, args.steps))
-    if True:
-        for it in range(e2e_steps + 10):
-            if it == 10:
-                barrier(dist)
-                stream.synchronize()
-                x0 = torch.cuda.Event(enable_timing=True)
-                x0.record(stream)
-            stt = states[it % copies]
-            for name, t in host_in.items():
-                getattr(stt, name).copy_(t, non_blocking=True)
-            stt.append(nk, stream)
-            stt.attend(nk, stream)
-            host_out.copy_(stt.o16, non_blocking=True)
-        x1 = torch.cuda.Event(enable_timing=True)
-        x1.record(stream)
+    for it_ in range(e2e_steps + 10):
+        if it_ == 10:
+            barrier(dist)
+            stream.synchronize()
+            x0 = torch.cuda.Event(enable_timing=True)
+            x0.record(stream)
+        stt = states[it_ % copies]
+        stt.stage.copy_(host_stage, non_blocking=True)
+        stt.append(nk, stream)
+        stt.attend(nk, stream)
+        host_out.copy_(stt.o16, non_blocking=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(x0.elapsed_time(x1) / e2e_steps, dist)
+    del g_step, g_att, states
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations' kernels: long-context decode and the
+    # mixed chunked-prefill batch
+    long_rec = long_decode_record(stream, clocks, 1)
+    mixed_rec = mixed_record(stream, clocks, 2)
+    clocks.stop()
 
     peak, peak_kind = peaks()
     achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
@@ -437,13 +605,17 @@ def run_ours(args, rank, world, dist):
             "algorithmic_bytes": app_bytes,
             "traffic": profiled_traffic("quantize_append_kernel<128>", "append_sweep"),
         },
+        "long_decode": long_rec,
+        "mixed_prefill_decode": mixed_rec,
         "e2e": {
             "value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(e2e_ms, 5),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "copies_per_step": "1 H2D (packed inputs) + 1 D2H",
         },
-        "gpu_launches": 2 * args.steps,  # append, decode attention
-        "clocks": clocks.summary(),
+        # timed region: append + decode attention per step
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(0),
     }
     return result
 

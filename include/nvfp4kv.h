@@ -33,7 +33,8 @@
  *
  * Conventions for every entry point:
  *   - All pointers are caller-owned DEVICE memory unless stated; the library
- *     never allocates device memory and never synchronizes the stream.
+ *     never allocates device memory and never synchronizes the stream (the
+ *     status read-back calls excepted, which say so).
  *   - Work is enqueued on `stream` (cudaStream_t; NULL = legacy default).
  *   - Host-side validation failures return a negative status and launch
  *     nothing. A CUDA launch error returns NVFP4_ERR_CUDA. Device-side faults
@@ -67,7 +68,10 @@ typedef enum {
   NVFP4_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad shape */
   NVFP4_ERR_UNSUPPORTED = -2, /* valid but not built: head_size, block_size, GQA group */
   NVFP4_ERR_CUDA = -3,        /* kernel launch / CUDA runtime error */
-  NVFP4_ERR_WORKSPACE = -4    /* workspace null or smaller than required */
+  NVFP4_ERR_WORKSPACE = -4,   /* workspace null or smaller than required */
+  NVFP4_ERR_DEVICE_BOUNDS = -5, /* read back: a kernel skipped an out-of-range
+                                   slot, block id or query range */
+  NVFP4_ERR_DEVICE_TIMEOUT = -6 /* read back: a bounded pipeline wait gave up */
 } nvfp4_status;
 
 /* Bits of the device status word (see nvfp4_paged_attention's workspace and
@@ -75,6 +79,8 @@ typedef enum {
 #define NVFP4_DEV_BAD_SLOT 0x1u    /* slot >= num_blocks*block_size (token skipped) */
 #define NVFP4_DEV_BAD_BLOCK 0x2u   /* block id outside [0, num_blocks) (page skipped) */
 #define NVFP4_DEV_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
+#define NVFP4_DEV_BAD_QLEN 0x8u    /* a query range longer than max_q_len (rows
+                                      past max_q_len left unwritten) */
 
 /* Row width in bytes, head_size/2 + head_size/16 ("FlashInfer backend adds
  * end-to-end NVFP4 KV cache support", get_kv_cache_shape, the
@@ -205,10 +211,13 @@ NVFP4KV_API int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
  * (nvfp4_paged_attention_workspace_size) exceeds it return
  * NVFP4_ERR_WORKSPACE. The first call on a device looks up the array's
  * device address on that device (make that first call before any stream
- * capture). Each call clears the array's status word and arrival counters
- * on `stream` first; all calls share the one array, so calls that may
- * overlap on the GPU (unordered streams) race and must not be made. The
- * call never calls cudaMalloc, cudaFree or any allocating routine. */
+ * capture; the look-up is repeated if the device's context is ever
+ * re-created). Each call clears the array's arrival counters on `stream`
+ * first; its status word is sticky across calls, like a workspace's, and is
+ * read (and optionally cleared) with nvfp4_paged_attention_noalloc_status.
+ * All calls share the one array, so calls that may overlap on the GPU
+ * (unordered streams) race and must not be made. The call never calls
+ * cudaMalloc, cudaFree or any allocating routine. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)12 << 20)
 NVFP4KV_API int nvfp4_paged_attention_noalloc(
     const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
@@ -217,6 +226,38 @@ NVFP4KV_API int nvfp4_paged_attention_noalloc(
     const int32_t* seq_lens, const int32_t* qo_indptr, int32_t num_seqs, int32_t max_q_len,
     const float* kv_scales, float sm_scale, uint8_t* o_fp8, const float* o_scale,
     void* o_bf16, float* o_f32, nvfp4_stream_t stream);
+
+/* nvfp4_read_device_status for the status word of the allocation-free
+ * entry point's scratch array on the current device (same synchronization,
+ * clearing and return codes). */
+NVFP4KV_API int nvfp4_paged_attention_noalloc_status(uint32_t* host_bits, int clear,
+                                                     nvfp4_stream_t stream);
+
+/* Device status read-back (the status reporting of the method statement's
+ * C ABI; the pages raise errors at start-up only). Copies the 4-byte device
+ * status word at `status_word` (a workspace's first 4 bytes, or the word given
+ * to nvfp4_quantize_append_paged as device_status) to the host after the work
+ * already enqueued on `stream`, SYNCHRONIZES the stream, optionally clears the
+ * word (clear != 0, enqueued on `stream`), and stores the bits in *host_bits
+ * (may be NULL). Returns NVFP4_ERR_DEVICE_TIMEOUT if NVFP4_DEV_TIMEOUT is set,
+ * else NVFP4_ERR_DEVICE_BOUNDS if any of NVFP4_DEV_BAD_SLOT / _BAD_BLOCK /
+ * _BAD_QLEN is set, else NVFP4_OK (or a CUDA / argument error). Not for use
+ * inside stream capture. */
+NVFP4KV_API int nvfp4_read_device_status(const uint32_t* status_word, uint32_t* host_bits,
+                                         int clear, nvfp4_stream_t stream);
+
+/* The status code nvfp4_read_device_status returns for a set of NVFP4_DEV_*
+ * bits. Pure host function. */
+NVFP4KV_API int nvfp4_status_from_bits(uint32_t bits);
+
+/* Self-test of the kernels' bounded waits (no counterpart in the pages; the
+ * failure-detection contract above). Launches one block that arms a
+ * shared-memory barrier for 16 bytes that no copy will deliver and waits on it
+ * with at most `polls` polls (1 .. 2^24); when the wait gives up it ORs
+ * NVFP4_DEV_TIMEOUT into the device word *status_word and returns. Nothing is
+ * in flight when the block exits, so the context stays usable. */
+NVFP4KV_API int nvfp4_wait_timeout_probe(uint32_t* status_word, int32_t polls,
+                                         nvfp4_stream_t stream);
 
 /* Static description of a status code. */
 NVFP4KV_API const char* nvfp4_status_string(int status);

@@ -22,10 +22,13 @@ NVFP4_ERR_INVALID_ARG = -1
 NVFP4_ERR_UNSUPPORTED = -2
 NVFP4_ERR_CUDA = -3
 NVFP4_ERR_WORKSPACE = -4
+NVFP4_ERR_DEVICE_BOUNDS = -5
+NVFP4_ERR_DEVICE_TIMEOUT = -6
 
 DEV_BAD_SLOT = 0x1
 DEV_BAD_BLOCK = 0x2
 DEV_TIMEOUT = 0x4
+DEV_BAD_QLEN = 0x8
 NVFP4_ATTN_METADATA_READY = 0x1
 
 
@@ -76,6 +79,15 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_paged_attention_noalloc.restype = ctypes.c_int
     L.nvfp4_dequantize_paged.argtypes = [P, i64, i32, i32, i32, P, i64, P, P, P]
     L.nvfp4_dequantize_paged.restype = ctypes.c_int
+    L.nvfp4_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
+    L.nvfp4_read_device_status.restype = ctypes.c_int
+    L.nvfp4_status_from_bits.argtypes = [ctypes.c_uint32]
+    L.nvfp4_status_from_bits.restype = ctypes.c_int
+    L.nvfp4_paged_attention_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_uint32),
+                                                       ctypes.c_int, P]
+    L.nvfp4_paged_attention_noalloc_status.restype = ctypes.c_int
+    L.nvfp4_wait_timeout_probe.argtypes = [P, i32, P]
+    L.nvfp4_wait_timeout_probe.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -155,9 +167,41 @@ def alloc_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_siz
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def read_device_status(status_word: torch.Tensor, clear: bool = False,
+                       stream: Optional[torch.cuda.Stream] = None):
+    """(status code, DEV_* bits) of a device status word -- a workspace (its
+    first 4 bytes) or a writer's device_status -- through
+    nvfp4_read_device_status (synchronizes the stream; clear resets it)."""
+    bits = ctypes.c_uint32(0)
+    st = lib().nvfp4_read_device_status(_ptr(status_word), ctypes.byref(bits), int(clear),
+                                        _stream(stream))
+    if st not in (NVFP4_OK, NVFP4_ERR_DEVICE_BOUNDS, NVFP4_ERR_DEVICE_TIMEOUT):
+        _check(st, "nvfp4_read_device_status")
+    return st, int(bits.value)
+
+
 def workspace_status(workspace: torch.Tensor) -> int:
     """Device status bits (DEV_*) recorded in a workspace (synchronizes)."""
-    return int(workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
+    return read_device_status(workspace)[1]
+
+
+def noalloc_status(clear: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """(status code, DEV_* bits) of the allocation-free entry point's scratch
+    status word on the current device (synchronizes; clear resets it)."""
+    bits = ctypes.c_uint32(0)
+    st = lib().nvfp4_paged_attention_noalloc_status(ctypes.byref(bits), int(clear),
+                                                    _stream(stream))
+    if st not in (NVFP4_OK, NVFP4_ERR_DEVICE_BOUNDS, NVFP4_ERR_DEVICE_TIMEOUT):
+        _check(st, "nvfp4_paged_attention_noalloc_status")
+    return st, int(bits.value)
+
+
+def wait_timeout_probe(status_word: torch.Tensor, polls: int = 1000,
+                       stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Launch the bounded-wait self-test: a wait that nothing completes gives up
+    after `polls` polls and ORs DEV_TIMEOUT into status_word (int32 device)."""
+    _check(lib().nvfp4_wait_timeout_probe(_ptr(status_word), polls, _stream(stream)),
+           "nvfp4_wait_timeout_probe")
 
 
 def _attention_dims(q, cache, block_table, seq_lens, qo_indptr, o_fp8, o_bf16, o_f32):

@@ -1,5 +1,6 @@
 // C ABI of libnvfp4kv: host-side validation, then kernel launches on the
 // caller's stream. See include/nvfp4kv.h for the contract of each call.
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include "../../include/nvfp4kv.h"
@@ -16,6 +17,32 @@ thread_local const char* g_last_error = "no error";
 }  // namespace
 
 namespace nvfp4kv {
+
+cudaError_t current_context_id(unsigned long long* id) {
+  struct Fns {
+    PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    PFN_cuCtxGetId_v12000 get_id = nullptr;
+  };
+  static const Fns fns = [] {
+    Fns f;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    return f;
+  }();
+  *id = 0;
+  if (!fns.get_current || !fns.get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (fns.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+  if (!ctx) return cudaSuccess;
+  return fns.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorUnknown;
+}
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return NVFP4_OK;
@@ -120,6 +147,10 @@ const char* nvfp4_status_string(int status) {
       return "CUDA error";
     case NVFP4_ERR_WORKSPACE:
       return "workspace missing or too small";
+    case NVFP4_ERR_DEVICE_BOUNDS:
+      return "a kernel skipped an out-of-range slot, block id or query range";
+    case NVFP4_ERR_DEVICE_TIMEOUT:
+      return "a kernel's bounded pipeline wait gave up";
     default:
       return "unknown status";
   }
@@ -199,6 +230,36 @@ int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_
   a.workspace = workspace;
   a.flags = flags;
   return nvfp4kv::launch_attention(a, (cudaStream_t)stream);
+}
+
+int nvfp4_status_from_bits(uint32_t bits) {
+  if (bits & NVFP4_DEV_TIMEOUT) return NVFP4_ERR_DEVICE_TIMEOUT;
+  if (bits & (NVFP4_DEV_BAD_SLOT | NVFP4_DEV_BAD_BLOCK | NVFP4_DEV_BAD_QLEN))
+    return NVFP4_ERR_DEVICE_BOUNDS;
+  return NVFP4_OK;
+}
+
+int nvfp4_read_device_status(const uint32_t* status_word, uint32_t* host_bits, int clear,
+                             nvfp4_stream_t stream) {
+  if (!status_word || !aligned(status_word, 4)) return NVFP4_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t bits = 0;
+  int st = cuda_status(cudaMemcpyAsync(&bits, status_word, sizeof(bits), cudaMemcpyDeviceToHost, s));
+  if (st != NVFP4_OK) return st;
+  st = cuda_status(cudaStreamSynchronize(s));
+  if (st != NVFP4_OK) return st;
+  if (clear && bits) {
+    st = cuda_status(cudaMemsetAsync(const_cast<uint32_t*>(status_word), 0, sizeof(bits), s));
+    if (st != NVFP4_OK) return st;
+  }
+  if (host_bits) *host_bits = bits;
+  return nvfp4_status_from_bits(bits);
+}
+
+int nvfp4_wait_timeout_probe(uint32_t* status_word, int32_t polls, nvfp4_stream_t stream) {
+  if (!status_word || !aligned(status_word, 4) || polls < 1 || polls > (1 << 24))
+    return NVFP4_ERR_INVALID_ARG;
+  return cuda_status(nvfp4kv::launch_wait_timeout_probe(status_word, polls, (cudaStream_t)stream));
 }
 
 int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks, int32_t block_size,

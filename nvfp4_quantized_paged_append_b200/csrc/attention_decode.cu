@@ -46,6 +46,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 namespace nvfp4kv {
 
 namespace {
@@ -653,6 +655,9 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
       const int q0 = a.qo_indptr ? a.qo_indptr[b] : b;
       const int ql = a.qo_indptr ? a.qo_indptr[b + 1] - q0 : 1;
       const int L = a.seq_lens[b];
+      // a query range longer than the host's bound is not fully served by the
+      // prefill grid (sized from max_q_len): flagged, by block 0 only
+      if (ql > max(1, a.max_q_len) && blockIdx.x == 0) atomicOr(status, kDevBadQlen);
       const int pages = min(a.max_blocks_per_seq, max(1, (L + BS - 1) / BS));
       const int ub = (pages + U - 1) / U;
       val = (ql == 1) ? ub * Hkv : 0;
@@ -1095,16 +1100,19 @@ static cudaError_t encode_page_rows(CUtensorMap* map, const uint8_t* cache, int6
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Per-device launch facts, looked up once (outside any stream capture: the
-// first call on a device should be an eager one).
+// Per-device launch facts, looked up once per (device, context) under a lock
+// (outside any stream capture: the first call on a device should be an eager
+// one).
 struct DeviceFacts {
   int sms = 0;
+  unsigned long long ctx[2] = {0, 0};  // context the attribute was set in, per DUP
   bool smem_attr_set[2] = {false, false};
 };
 
 template <int D, int BS, bool DUP>
 static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) {
   using S = DecodeShape<D, BS>;
+  static std::mutex facts_mutex;
   static DeviceFacts facts[64];
   const int G = a.num_q_heads / a.num_kv_heads;
   const int nw = S::warps_for(a.num_seqs, G);
@@ -1114,26 +1122,36 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  DeviceFacts& f = facts[dev & 63];
-  if (!f.smem_attr_set[DUP]) {
-    // allow the largest dynamic size the device permits beside the static part
-    int optin = 0;
-    err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (err != cudaSuccess) return err;
-    cudaFuncAttributes fa;
-    err = cudaFuncGetAttributes(&fa, kern);
-    if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               optin - (int)fa.sharedSizeBytes);
-    if (err != cudaSuccess) return err;
-    err = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return err;
-    f.smem_attr_set[DUP] = true;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  unsigned long long ctx = 0;
+  err = current_context_id(&ctx);
+  if (err != cudaSuccess) return err;
+  int sms = 0;
+  {
+    std::lock_guard<std::mutex> lock(facts_mutex);
+    DeviceFacts& f = facts[dev];
+    if (!f.smem_attr_set[DUP] || ctx == 0 || f.ctx[DUP] != ctx) {
+      // allow the largest dynamic size the device permits beside the static part
+      int optin = 0;
+      err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+      if (err != cudaSuccess) return err;
+      cudaFuncAttributes fa;
+      err = cudaFuncGetAttributes(&fa, kern);
+      if (err != cudaSuccess) return err;
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 optin - (int)fa.sharedSizeBytes);
+      if (err != cudaSuccess) return err;
+      err = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev);
+      if (err != cudaSuccess) return err;
+      f.smem_attr_set[DUP] = true;
+      f.ctx[DUP] = ctx;
+    }
+    sms = f.sms;
   }
   int per_sm = 1;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nw * 32, smem);
   if (err != cudaSuccess) return err;
-  int grid = f.sms * max(1, per_sm);
+  int grid = sms * max(1, per_sm);
   if (grid * nw > kDecodeWarps) grid = kDecodeWarps / nw;
   AttentionArgs ag = a;
   if constexpr (S::kGather) {

@@ -13,6 +13,8 @@
 // cooperative dequant into f16 tiles in shared memory (exact: E2M1 * E4M3 has
 // at most 6 significant bits), then mma.m16n8k16 for S = Q K^T and O += P V
 // with fp32 accumulators and an exp2-domain online softmax.
+#include <mutex>
+
 #include "nvfp4kv_device.cuh"
 #include "nvfp4kv_launch.h"
 
@@ -58,6 +60,8 @@ __global__ void __launch_bounds__(kPWarps * 32) prefill_attention_kernel(const A
   const int q_begin = a.qo_indptr[b];
   const int q_len = a.qo_indptr[b + 1] - q_begin;
   if (q_len <= 1) return;  // decode rows are served by the decode kernel
+  if (q_len > (int)gridDim.x * tpt && blockIdx.x == 0 && threadIdx.x == 0)
+    atomicOr(reinterpret_cast<uint32_t*>(a.workspace), kDevBadQlen);  // rows beyond the grid
   const int qtok0 = blockIdx.x * tpt;
   if (qtok0 >= q_len) return;
   const int L = a.seq_lens[b];
@@ -296,14 +300,23 @@ static cudaError_t launch_prefill_t(const AttentionArgs& a, cudaStream_t stream)
   using S = PrefillShape<D, BS>;
   const size_t smem = S::smem_bytes();
   auto kern = prefill_attention_kernel<D, BS>;
-  static bool attr_set[64] = {false};
+  // the attribute is set once per (device, context), under a lock
+  static std::mutex attr_mutex;
+  static unsigned long long attr_ctx[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (!attr_set[dev & 63]) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    attr_set[dev & 63] = true;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  unsigned long long ctx = 0;
+  err = current_context_id(&ctx);
+  if (err != cudaSuccess) return err;
+  {
+    std::lock_guard<std::mutex> lock(attr_mutex);
+    if (ctx == 0 || attr_ctx[dev] != ctx) {
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      attr_ctx[dev] = ctx;
+    }
   }
   const int G = a.num_q_heads / a.num_kv_heads;
   const int tpt = kRows / G;

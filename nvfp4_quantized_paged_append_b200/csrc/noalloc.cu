@@ -13,12 +13,15 @@
 // every GPU that loads this library holds that much memory until the process
 // exits. Host code cannot use the array's name as a device address, so the
 // first call on each device looks the address up with cudaGetSymbolAddress
-// (with that device current) and caches it; do that first call outside any
-// stream capture. All calls on a device share the array and the array keeps
-// whatever the previous call left in it, so each call clears the part that
-// must start at zero (status word and arrival counters) on its stream
-// before the kernels run. Calls that overlap on the GPU (different streams,
-// no ordering between them) race on the array and must not be issued.
+// (with that device current) and keeps it for that device's context; do that
+// first call outside any stream capture. If the context is re-created (after
+// cudaDeviceReset), the next call looks the address up again. All calls on a
+// device share the array and the array keeps whatever the previous call left
+// in it, so each call clears the part that must start at zero (the arrival
+// counters) on its stream before the kernels run. The status word is sticky,
+// as in a caller's workspace: nvfp4_paged_attention_noalloc_status reads and
+// optionally clears it. Calls that overlap on the GPU (different streams, no
+// ordering between them) race on the array and must not be issued.
 #include <mutex>
 
 #include "../../include/nvfp4kv.h"
@@ -39,19 +42,27 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array on the current device, looked up once
+// per (device, context).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned long long ctx = 0;
+  err = nvfp4kv::current_context_id(&ctx);
+  if (err != cudaSuccess) return err;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_nvfp4_scratch);
     if (err != cudaSuccess) return err;
+    // the look-up makes the context current if none was
+    if (ctx == 0 && nvfp4kv::current_context_id(&ctx) != cudaSuccess) ctx = 0;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -84,12 +95,20 @@ int nvfp4_paged_attention_noalloc(const void* q, int64_t q_token_stride, int64_t
   int cst = nvfp4kv::cuda_status(scratch_address(&scratch));
   if (cst != NVFP4_OK) return cst;
   cudaStream_t s = (cudaStream_t)stream;
-  // status word + arrival counters must start at zero; partial slots are
-  // always written before they are read
-  cst = nvfp4kv::cuda_status(cudaMemsetAsync(scratch, 0, wl.partials_off, s));
+  // the arrival counters must start at zero; partial slots are always written
+  // before they are read; the status word (bytes 0..3) is left as it is
+  cst = nvfp4kv::cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(scratch) + wl.counters_off, 0,
+                                             wl.partials_off - wl.counters_off, s));
   if (cst != NVFP4_OK) return cst;
   a.workspace = scratch;
   return nvfp4kv::launch_attention(a, s);
+}
+
+int nvfp4_paged_attention_noalloc_status(uint32_t* host_bits, int clear, nvfp4_stream_t stream) {
+  void* scratch = nullptr;
+  const int cst = nvfp4kv::cuda_status(scratch_address(&scratch));
+  if (cst != NVFP4_OK) return cst;
+  return nvfp4_read_device_status(static_cast<const uint32_t*>(scratch), host_bits, clear, stream);
 }
 
 }  // extern "C"

@@ -19,6 +19,7 @@ namespace nvfp4kv {
 constexpr uint32_t kDevBadSlot = 0x1u;
 constexpr uint32_t kDevBadBlock = 0x2u;
 constexpr uint32_t kDevTimeout = 0x4u;
+constexpr uint32_t kDevBadQlen = 0x8u;
 constexpr uint32_t kAttnMetadataReady = 0x1u;  // NVFP4_ATTN_METADATA_READY
 
 // Wait until the grids this one depends on (programmatic dependent launch)
@@ -204,8 +205,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for phase `parity` of `bar` to complete. Returns false (and
 // the caller reports NVFP4_DEV_TIMEOUT) if it did not complete in time.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  for (int i = 0; i < kMaxWaitIters; ++i)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  int max_iters = kMaxWaitIters) {
+  for (int i = 0; i < max_iters; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

@@ -89,9 +89,18 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int num_seqs, int nu
   return w;
 }
 
+// Unique id of the CUDA context current on the calling thread (0 if none is
+// current yet). Per-device launch caches are keyed on it, so set-up done for a
+// context that was since destroyed (cudaDeviceReset) is done again.
+cudaError_t current_context_id(unsigned long long* id);
+
 cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t stream);
 cudaError_t launch_dequantize_paged(const DequantArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_attention(const AttentionArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attention(const AttentionArgs& a, cudaStream_t stream);
+// A one-block kernel that arms an mbarrier for 16 bytes no copy will deliver,
+// waits on it with at most `polls` polls and ORs kDevTimeout into *status when
+// the wait gives up (nothing is in flight when it returns).
+cudaError_t launch_wait_timeout_probe(uint32_t* status, int polls, cudaStream_t stream);
 
 }  // namespace nvfp4kv

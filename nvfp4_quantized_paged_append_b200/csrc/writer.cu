@@ -23,8 +23,16 @@ namespace nvfp4kv {
 // code, no rounding threshold of the E2M1 grid lies between them, and the
 // conversion is monotone, so fl32(x / S) has that code as well. Otherwise
 // (x / S within ~1e-6 of a threshold, exact ties included) the quotient is
-// formed with IEEE division. S must be a positive normal number.
+// formed with IEEE division. S must be a positive normal number; above
+// 2^100 the reciprocal nears the subnormal range, where its 1-ulp bound no
+// longer holds, so such scales always divide.
 __device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S) {
+  if (S > 1.2676506e30f) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
+    return f32x8_to_e2m1x8(q);
+  }
   float r;
   asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(S));
   float lo[8], hi[8];
@@ -189,6 +197,23 @@ cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t str
       return cudaErrorInvalidValue;
   }
 #undef NVFP4_WRITER_CASE
+  return cudaGetLastError();
+}
+
+// Bounded-wait check: the barrier expects 16 bytes that no copy delivers, so
+// the wait must give up after `polls` polls and report kDevTimeout. No copy is
+// ever issued, so nothing is in flight when the block exits.
+__global__ void wait_timeout_probe_kernel(uint32_t* status, int polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_arrive_expect_tx(&bar, 16);
+  if (!mbar_wait_bounded(&bar, 0u, polls)) atomicOr(status, kDevTimeout);
+}
+
+cudaError_t launch_wait_timeout_probe(uint32_t* status, int polls, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, polls);
   return cudaGetLastError();
 }
 

@@ -115,6 +115,19 @@ class PagedWorkload:
             total += int(np.clip(p + 1, 0, None).sum())
         return total * self.num_q_heads * 4 * self.head_size
 
+    def subset(self, seqs: Sequence[int]):
+        """(workload over the listed sequences, int64 indices of their query
+        tokens in this workload's q). The subset shares this workload's cache
+        (same num_blocks and block ids); its tensor data is not redrawn."""
+        seqs = [int(b) for b in seqs]
+        ind = self.qo_indptr
+        tok = np.concatenate([np.arange(ind[b], ind[b + 1], dtype=np.int64) for b in seqs])
+        sub = dataclasses.replace(self, name=f"{self.name}[{len(seqs)} seqs]",
+                                  seq_lens=self.seq_lens[seqs].copy(),
+                                  q_lens=self.q_lens[seqs].copy(),
+                                  block_table=np.ascontiguousarray(self.block_table[seqs]))
+        return sub, tok
+
     def slots_for_seq(self, b: int, start: int = 0, stop: Optional[int] = None) -> np.ndarray:
         """Cache slots of tokens start..stop-1 of sequence b (int64)."""
         stop = int(self.seq_lens[b]) if stop is None else stop

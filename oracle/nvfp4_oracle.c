@@ -24,7 +24,8 @@
  *        attention in fp32 online softmax is defined here as plain fp64
  *        softmax attention over the dequantized cache.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent (the pages above fix only the shapes,
+ * the packing and the scale formats; the method statement fixes the rounding):
  *   - element 2j sits in the LOW nibble of byte j, 2j+1 in the high nibble;
  *   - a row is [head_size/2 data bytes][head_size/16 scale bytes];
  *   - s32 = fl32(amax / fl32(6*g)); sb = E4M3_RNE_satfinite(s32);

@@ -37,9 +37,35 @@ def test_full_dim(L):
 
 
 def test_status_strings(L):
-    for s in (0, -1, -2, -3, -4):
-        assert nk.status_string(s)
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert nk.status_string(s) and nk.status_string(s) != "unknown status"
     assert nk.status_string(-99) == "unknown status"
+
+
+def test_status_from_device_bits(L):
+    """Device status bits map to the read-back codes: a timeout outranks the
+    bounds bits; no bit is NVFP4_OK."""
+    f = L.nvfp4_status_from_bits
+    assert f(0) == nk.NVFP4_OK
+    for b in (nk.DEV_BAD_SLOT, nk.DEV_BAD_BLOCK, nk.DEV_BAD_QLEN,
+              nk.DEV_BAD_SLOT | nk.DEV_BAD_BLOCK):
+        assert f(b) == nk.NVFP4_ERR_DEVICE_BOUNDS
+    for b in (nk.DEV_TIMEOUT, nk.DEV_TIMEOUT | nk.DEV_BAD_BLOCK):
+        assert f(b) == nk.NVFP4_ERR_DEVICE_TIMEOUT
+
+
+def test_status_readback_and_probe_validation(L):
+    """Null or misaligned status words and out-of-range poll limits are
+    rejected before any CUDA call."""
+    bits = ctypes.c_uint32(7)
+    assert L.nvfp4_read_device_status(None, ctypes.byref(bits), 0, None) == nk.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_read_device_status(ctypes.c_void_p(0x1002), None, 0, None) == \
+        nk.NVFP4_ERR_INVALID_ARG
+    assert bits.value == 7                                   # untouched on rejection
+    assert L.nvfp4_wait_timeout_probe(None, 100, None) == nk.NVFP4_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x1000)
+    assert L.nvfp4_wait_timeout_probe(fake, 0, None) == nk.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_wait_timeout_probe(fake, (1 << 24) + 1, None) == nk.NVFP4_ERR_INVALID_ARG
 
 
 def _append(L, **kw):

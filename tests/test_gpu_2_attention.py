@@ -121,13 +121,54 @@ def test_repeat_calls_identical_and_workspace_reusable():
 
 
 def test_bad_block_id_flagged_no_fault():
+    """A planted out-of-range block id is skipped (no fault) and reported through
+    the C ABI's status read-back as NVFP4_ERR_DEVICE_BOUNDS; clearing resets it."""
     w = wl.custom_workload("badblk", 5, 8, 2, 128, 16, [40, 70])
     scales = wl.global_scales(w, DEV)
     cache = build_gpu_cache(w, scales, DEV)
     w.block_table[1, 2] = w.num_blocks + 1000   # out of range
     out = run_gpu_attention(w, cache, scales, DEV)
-    assert nk.workspace_status(out[3]) & nk.DEV_BAD_BLOCK
+    st, bits = nk.read_device_status(out[3], clear=True)
+    assert st == nk.NVFP4_ERR_DEVICE_BOUNDS and bits & nk.DEV_BAD_BLOCK
+    assert nk.read_device_status(out[3]) == (nk.NVFP4_OK, 0)
     assert torch.isfinite(out[2]).all()
+
+
+def test_query_range_beyond_max_q_len_flagged():
+    """A prefill range longer than the host's max_q_len bound leaves rows beyond
+    the launched grid unwritten and raises DEV_BAD_QLEN (read back through the
+    C ABI)."""
+    w = wl.custom_workload("badqlen", 6, 8, 2, 128, 16, [300, 90], [200, 1])
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    q = wl.queries(w, DEV)
+    o8 = torch.zeros((w.num_q_tokens, w.num_q_heads, w.head_size), dtype=torch.uint8, device=DEV)
+    ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, DEV)
+    nk.paged_attention(q, cache, torch.from_numpy(w.block_table).to(DEV),
+                       torch.from_numpy(w.seq_lens).to(DEV),
+                       torch.tensor([scales[0], scales[1]], device=DEV), o8,
+                       torch.tensor([scales[2]], device=DEV), ws,
+                       qo_indptr=torch.from_numpy(w.qo_indptr).to(DEV), max_q_len=16)
+    st, bits = nk.read_device_status(ws)
+    assert st == nk.NVFP4_ERR_DEVICE_BOUNDS and bits & nk.DEV_BAD_QLEN
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """The bounded-wait self-test: a barrier wait that no copy completes gives up
+    after its poll limit, the kernel returns, DEV_TIMEOUT reads back as
+    NVFP4_ERR_DEVICE_TIMEOUT, and the context still runs attention correctly."""
+    word = torch.zeros(1, dtype=torch.int32, device=DEV)
+    nk.wait_timeout_probe(word, polls=2000)
+    st, bits = nk.read_device_status(word, clear=True)
+    assert st == nk.NVFP4_ERR_DEVICE_TIMEOUT and bits == nk.DEV_TIMEOUT
+    assert nk.read_device_status(word) == (nk.NVFP4_OK, 0)
+    w = wl.make_workload("tiny_decode")
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    out = run_gpu_attention(w, cache, scales, DEV)
+    assert nk.read_device_status(out[3]) == (nk.NVFP4_OK, 0)
+    case = oracle_case(w, range(w.num_seqs), scales, DEV)
+    _compare(w, scales, out[:3], case, run_oracle(case, scales))
 
 
 def test_output_scale_and_sm_scale_arguments():

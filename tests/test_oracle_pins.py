@@ -347,3 +347,28 @@ def test_attention_special_cases():
                                         np.array([0, 3], np.int32), 1.0, 1.0)
     assert np.all(o64[0] == 0) and np.any(o64[1] != 0) and np.any(o64[2] != 0)
     assert np.array_equal(o64[1, 0], xhat[2, 1, 0, 0])          # row 1 sees key 0 only
+
+
+@pytest.mark.parametrize("D,bs,H", [(64, 16, 2), (128, 32, 3), (256, 16, 1)])
+def test_dequantize_paged_scales_and_block_list(D, bs, H):
+    """The paged dequantize helper ("FlashInfer NVFP4 KV serving on pre-SM100
+    GPUs", quick answer) on a hand-packed multi-block cache: K pages take
+    k_scale and V pages v_scale (two different non-unit values), and out[i]
+    holds the pages of block_ids[i] for a repeated, unordered id list.
+    Expected bits: the hand-packed xhat (exact in fp32), times g in fp32,
+    rounded to bf16 by torch."""
+    rng = np.random.default_rng(D + bs + H)
+    NB = 5
+    cache, xhat = _hand_cache(rng, NB, H, bs, D)
+    ids = np.array([3, 0, 3, 4, 1], np.int32)
+    gk, gv = float(np.float32(0.37)), float(np.float32(2.5))
+    got = oracle.dequantize_paged(cache, ids, gk, gv)
+    x32 = torch.from_numpy(xhat[ids].astype(np.float32))            # exact: <= 6 significant bits
+    assert np.array_equal(x32.double().numpy(), xhat[ids])
+    g = torch.tensor([gk, gv], dtype=torch.float32).view(1, 2, 1, 1, 1)
+    want = (x32 * g).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert got.shape == (len(ids), 2, H, bs, D)
+    assert np.array_equal(got, want)
+    # a K/V scale swap or a scale dropped would change the bits
+    swapped = (x32 * g.flip(1)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert not np.array_equal(got, swapped)

@@ -43,6 +43,7 @@ def test_noalloc_matches_workspace_entry_point(make):
     kvs = torch.tensor([scales[0], scales[1]], dtype=torch.float32, device=DEV)
     osc = dev_scalar(scales[2])
 
+    nk.noalloc_status(clear=True)        # the status word is sticky across calls
     ref8, ref16, ref32 = _outputs(w)
     ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, DEV)
     nk.paged_attention(q, cache, bt, sl, kvs, ref8, osc, ws, qo_indptr=qo, max_q_len=w.max_q_len,
@@ -57,6 +58,27 @@ def test_noalloc_matches_workspace_entry_point(make):
         d = w.head_size
         check_rows(o32.cpu().numpy().reshape(-1, d), ref32.cpu().numpy().reshape(-1, d).astype(np.float64))
         check_fp8(o8.cpu().numpy(), ref8.cpu().numpy())
+        assert nk.noalloc_status() == (nk.NVFP4_OK, 0)
+
+
+def test_noalloc_reports_device_status():
+    """A planted out-of-range block id: the allocation-free call skips the page
+    like the workspace call does, and its status read-back reports it (then
+    clears it)."""
+    w = wl.custom_workload("noalloc_badblk", 5, 8, 2, 128, 16, [40, 70])
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    w.block_table[1, 2] = w.num_blocks + 1000
+    nk.noalloc_status(clear=True)
+    o8, o16, o32 = _outputs(w)
+    nk.paged_attention_noalloc(wl.queries(w, DEV), cache, torch.from_numpy(w.block_table).to(DEV),
+                               torch.from_numpy(w.seq_lens).to(DEV),
+                               torch.tensor([scales[0], scales[1]], device=DEV), o8,
+                               dev_scalar(scales[2]), o_f32=o32)
+    st, bits = nk.noalloc_status(clear=True)
+    assert st == nk.NVFP4_ERR_DEVICE_BOUNDS and bits & nk.DEV_BAD_BLOCK
+    assert nk.noalloc_status() == (nk.NVFP4_OK, 0)
+    assert torch.isfinite(o32).all()
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
