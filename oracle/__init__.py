@@ -53,6 +53,12 @@ def lib():
             P, i64, ctypes.c_int, P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             P, ctypes.c_int, P, P, ctypes.c_int, f32, f32, f64, f32, P, P, P]
         _lib.nvo_paged_attention.restype = None
+        _lib.nvo_act_sf_bytes.argtypes = [i64, i64, ctypes.c_int]
+        _lib.nvo_act_sf_bytes.restype = i64
+        _lib.nvo_act_sf_index.argtypes = [i64, i64, i64]
+        _lib.nvo_act_sf_index.restype = i64
+        _lib.nvo_quantize_activation.argtypes = [P, i64, i64, i64, f32, P, P, ctypes.c_int]
+        _lib.nvo_quantize_activation.restype = None
         del i32
     return _lib
 
@@ -164,3 +170,27 @@ def paged_attention(q, cache, block_table, seq_lens, qo_indptr, k_scale,
         _ptr(seq_lens), _ptr(qo_indptr), B, k_scale, v_scale, sm_scale, o_scale,
         _ptr(o64), _ptr(o8), _ptr(o16))
     return o64, o8, o16
+
+
+# ---------------------------------------------------------------- activations
+def act_sf_bytes(rows: int, cols: int, swizzled: bool) -> int:
+    return int(lib().nvo_act_sf_bytes(rows, cols, int(swizzled)))
+
+
+def act_sf_index(r: int, c: int, cols: int) -> int:
+    """Byte position of scale (row r, scale column c) in the swizzled layout."""
+    return int(lib().nvo_act_sf_index(r, c, cols))
+
+
+def quantize_activation(x, global_scale_inv, swizzled=True):
+    """bf16 bits uint16[rows][cols] -> (uint8[rows][cols/2] packed E2M1,
+    uint8 scales: swizzled flat array, or [rows][cols/16])."""
+    _need(x, np.uint16, "x")
+    rows, cols = x.shape
+    fp4 = np.zeros((rows, cols // 2), np.uint8)
+    n = act_sf_bytes(rows, cols, swizzled)
+    sf = np.zeros(n, np.uint8)
+    lib().nvo_quantize_activation(_ptr(x), rows, cols, cols, global_scale_inv, _ptr(fp4),
+                                  _ptr(sf), int(swizzled))
+    return fp4, (sf if swizzled else sf.reshape(rows, cols // 16))
+

@@ -361,3 +361,54 @@ void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
   free(row_seq);
   free(row_idx);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Activation quantizer with the block-scaled GEMM's scale-factor layout      */
+/* ------------------------------------------------------------------------ */
+
+/* [P3] "Move NVFP4 GEMM management into NvFp4LinearKernel", flashinfer.py and
+ * the CUTLASS linear kernel: scaled_fp4_quant(x, input_global_scale_inv,
+ * is_sf_swizzled_layout=True) turns the activations into packed E2M1 pairs
+ * plus one E4M3 scale per 16 values, and swizzle_blockscale rearranges scales
+ * for the block-scaled GEMM. The pages name both helpers without defining
+ * them; the readings taken here:
+ *   - the argument is the inverse global scale; g = fl32(1 / inv) (IEEE
+ *     division), and every row is then quantized exactly like a KV-cache row
+ *     (nvo_quantize_row): scale E4M3(amax / (6 g)), codes RNE onto E2M1;
+ *   - packed data: uint8 [rows][cols/2], element 2j in the low nibble;
+ *   - plain scales: uint8 [rows][cols/16];
+ *   - swizzled scales: rows padded to a multiple of 128 and scale columns to
+ *     a multiple of 4 (padding bytes 0); 512-byte tiles of 128 rows x 4 scale
+ *     columns, tile (r/128, c/4) at ((r/128) * (padded cols / 4) + c/4) * 512,
+ *     and inside a tile entry (r, c) at (r % 32) * 16 + ((r % 128) / 32) * 4
+ *     + c % 4 (the 32 x 4 x 4 interleave of the block-scaled MMA). */
+int64_t nvo_act_sf_bytes(int64_t rows, int64_t cols, int swizzled) {
+  int64_t c16 = cols / 16;
+  if (!swizzled) return rows * c16;
+  int64_t pr = (rows + 127) / 128 * 128, pc = (c16 + 3) / 4 * 4;
+  return pr * pc;
+}
+
+int64_t nvo_act_sf_index(int64_t r, int64_t c, int64_t cols) {
+  int64_t pc = (cols / 16 + 3) / 4 * 4;
+  int64_t tile = (r / 128) * (pc / 4) + c / 4;
+  return tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4;
+}
+
+void nvo_quantize_activation(const uint16_t* x, int64_t rows, int64_t cols,
+                             int64_t row_stride, float global_scale_inv,
+                             uint8_t* out_fp4, uint8_t* out_sf, int swizzled) {
+  float g = 1.0f / global_scale_inv; /* IEEE fp32 division */
+  int64_t c16 = cols / 16;
+  uint8_t* row = (uint8_t*)malloc((size_t)(cols / 2 + c16));
+  memset(out_sf, 0, (size_t)nvo_act_sf_bytes(rows, cols, swizzled));
+  for (int64_t r = 0; r < rows; ++r) {
+    nvo_quantize_row(x + r * row_stride, (int)cols, g, row);
+    memcpy(out_fp4 + r * (cols / 2), row, (size_t)(cols / 2));
+    for (int64_t c = 0; c < c16; ++c) {
+      int64_t at = swizzled ? nvo_act_sf_index(r, c, cols) : r * c16 + c;
+      out_sf[at] = row[cols / 2 + c];
+    }
+  }
+  free(row);
+}

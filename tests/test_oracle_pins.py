@@ -372,3 +372,57 @@ def test_dequantize_paged_scales_and_block_list(D, bs, H):
     # a K/V scale swap or a scale dropped would change the bits
     swapped = (x32 * g.flip(1)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert not np.array_equal(got, swapped)
+
+
+# ------------------------------------------------------------- activations
+def _golden_sf_positions():
+    rows = []
+    with open(os.path.join(GOLDEN, "sf_swizzle_positions.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                cols, r, c, pos = (int(x) for x in line.split()[:4])
+                rows.append((cols, r, c, pos))
+    return rows
+
+
+def test_activation_sf_positions_hand_worked():
+    """Swizzled scale positions worked by hand (tests/golden)."""
+    golden = _golden_sf_positions()
+    assert len(golden) >= 8
+    for cols, r, c, pos in golden:
+        assert oracle.act_sf_index(r, c, cols) == pos, (cols, r, c)
+
+
+@pytest.mark.parametrize("rows,cols", [(200, 96), (128, 64), (300, 4096 // 8), (1, 16)])
+def test_activation_sf_swizzle_vs_tile_transpose(rows, cols):
+    """The swizzled scales equal the plain [rows][cols/16] scales, zero-padded to
+    (128k rows, 4k columns), viewed as [row bands][4 groups of 32 rows][32]
+    [column tiles][4] and transposed to [band][column tile][32][4 groups][4]."""
+    rng = np.random.default_rng(rows + cols)
+    x = _bf16_bits(rng.standard_normal((rows, cols)).astype(np.float32) * 3)
+    inv = float(np.float32(448 * 6 / 9.0))
+    fp4_s, sf_s = oracle.quantize_activation(x, inv, swizzled=True)
+    fp4_p, sf_p = oracle.quantize_activation(x, inv, swizzled=False)
+    assert np.array_equal(fp4_s, fp4_p)
+    pr, pc = -(-rows // 128) * 128, -(-(cols // 16) // 4) * 4
+    pad = np.zeros((pr, pc), np.uint8)
+    pad[:rows, :cols // 16] = sf_p
+    want = pad.reshape(pr // 128, 4, 32, pc // 4, 4).transpose(0, 3, 2, 1, 4).reshape(-1)
+    assert np.array_equal(sf_s, want)
+
+
+def test_activation_rows_are_the_kv_row_codec():
+    """Each activation row is quantized exactly as a KV-cache row with the
+    global scale g = fl32(1 / inv): packed codes, then the row's scales."""
+    rng = np.random.default_rng(5)
+    rows, cols = 37, 256
+    x = _bf16_bits(rng.standard_normal((rows, cols)).astype(np.float32))
+    inv = float(np.float32(2688.0 / 4.25))
+    g = float(np.float32(1.0) / np.float32(inv))
+    fp4, sf = oracle.quantize_activation(x, inv, swizzled=False)
+    for r in range(rows):
+        row = oracle.quantize_row(np.ascontiguousarray(x[r]), g)
+        assert np.array_equal(fp4[r], row[:cols // 2]) and np.array_equal(sf[r], row[cols // 2:])
+    # g is the inverse of inv, not inv: the scales would change with inv itself
+    alt = oracle.quantize_row(np.ascontiguousarray(x[0]), inv)
+    assert not np.array_equal(sf[0], alt[cols // 2:])
