@@ -53,6 +53,10 @@ def lib():
             P, i64, ctypes.c_int, P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             P, ctypes.c_int, P, P, ctypes.c_int, f32, f32, f64, f32, P, P, P]
         _lib.nvo_paged_attention.restype = None
+        _lib.nvo_paged_attention_fmt.argtypes = _lib.nvo_paged_attention.argtypes + [ctypes.c_int]
+        _lib.nvo_paged_attention_fmt.restype = None
+        _lib.nvo_fp8kv_quantize_append_paged.argtypes = _lib.nvo_quantize_append_paged.argtypes
+        _lib.nvo_fp8kv_quantize_append_paged.restype = i64
         _lib.nvo_act_sf_bytes.argtypes = [i64, i64, ctypes.c_int]
         _lib.nvo_act_sf_bytes.restype = i64
         _lib.nvo_act_sf_index.argtypes = [i64, i64, i64]
@@ -146,12 +150,31 @@ def dequantize_paged(cache, block_ids, k_scale, v_scale):
 
 
 # ---------------------------------------------------------------- attention
+KV_NVFP4, KV_FP8 = 0, 1
+
+
+def fp8kv_quantize_append_paged(k, v, cache, slot_mapping, k_scale, v_scale, block_size):
+    """FP8-E4M3 writer on a numpy HND cache uint8[NB][2][Hkv][bs][D]:
+    E4M3_RNE_satfinite(fl32(x / g)) per element."""
+    _need(k, np.uint16, "k")
+    _need(v, np.uint16, "v")
+    _need(cache, np.uint8, "cache")
+    _need(slot_mapping, np.int64, "slot_mapping")
+    nb, two, hkv, bs, d = cache.shape
+    assert two == 2 and bs == block_size
+    T = slot_mapping.shape[0]
+    return lib().nvo_fp8kv_quantize_append_paged(
+        _ptr(k), _ptr(v), hkv * d, hkv * d, T, hkv, d, _ptr(cache), nb, bs,
+        _ptr(slot_mapping), k_scale, v_scale)
+
+
 def paged_attention(q, cache, block_table, seq_lens, qo_indptr, k_scale,
-                    v_scale, sm_scale=0.0, o_scale=1.0):
+                    v_scale, sm_scale=0.0, o_scale=1.0, kv_format=KV_NVFP4):
     """fp64 paged attention. Returns (o_f64, o_fp8, o_bf16_bits).
 
-    q: uint16 [Tq][Hq][D]; cache uint8[NB][2][Hkv][bs][F]; block_table int32
-    [B][max_blocks]; seq_lens int32 [B]; qo_indptr int32 [B+1] or None.
+    q: uint16 [Tq][Hq][D]; cache uint8[NB][2][Hkv][bs][F] (F = D/2 + D/16 for
+    NVFP4, D for FP8 rows); block_table int32 [B][max_blocks]; seq_lens int32
+    [B]; qo_indptr int32 [B+1] or None.
     """
     _need(q, np.uint16, "q")
     _need(cache, np.uint8, "cache")
@@ -165,10 +188,10 @@ def paged_attention(q, cache, block_table, seq_lens, qo_indptr, k_scale,
     o64 = np.zeros((tq, hq, d), np.float64)
     o8 = np.zeros((tq, hq, d), np.uint8)
     o16 = np.zeros((tq, hq, d), np.uint16)
-    lib().nvo_paged_attention(
+    lib().nvo_paged_attention_fmt(
         _ptr(q), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
         _ptr(seq_lens), _ptr(qo_indptr), B, k_scale, v_scale, sm_scale, o_scale,
-        _ptr(o64), _ptr(o8), _ptr(o16))
+        _ptr(o64), _ptr(o8), _ptr(o16), int(kv_format))
     return o64, o8, o16
 
 

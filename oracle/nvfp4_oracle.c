@@ -227,6 +227,21 @@ static double row_elem(const uint8_t* row, int head_size, int d) {
   return nvo_e2m1_decode(code) * nvo_e4m3_decode(row[head_size / 2 + d / 16]);
 }
 
+/* Row formats of the paged cache: NVFP4 (E2M1 pairs + E4M3 block scales,
+ * head_size/2 + head_size/16 bytes) or FP8 (one E4M3 byte per element,
+ * head_size bytes; the per-tensor k_scale / v_scale multiplies it). */
+enum { NVO_KV_NVFP4 = 0, NVO_KV_FP8 = 1 };
+
+static int64_t kv_row_bytes(int kv_format, int head_size) {
+  return kv_format == NVO_KV_FP8 ? (int64_t)head_size : nvo_full_dim(head_size);
+}
+
+/* Element d of a row without the global scale (exact in double). */
+static double kv_elem(int kv_format, const uint8_t* row, int head_size, int d) {
+  if (kv_format == NVO_KV_FP8) return nvo_e4m3_decode(row[d]);
+  return row_elem(row, head_size, d);
+}
+
 /* Standalone dequant of listed blocks: out[i] = bf16 pages of block
  * block_ids[i], layout bf16[num_block_ids][2][num_kv_heads][block_size]
  * [head_size]; value bf16_RNE(fl32(xhat * g)), g = k_scale for K pages and
@@ -271,17 +286,18 @@ void nvo_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
  * Outputs (each may be NULL): o_f64 [num_q_tokens][num_q_heads][head_size],
  * o_fp8 (E4M3 bytes), o_bf16 (bf16 bits), same shape.
  * Rows are independent; the loop over them is split across threads. */
-void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
-                         int num_q_heads, const uint8_t* cache,
-                         int64_t num_blocks, int block_size, int num_kv_heads,
-                         int head_size, const int32_t* block_table,
-                         int max_blocks_per_seq, const int32_t* seq_lens,
-                         const int32_t* qo_indptr, int num_seqs, float k_scale,
-                         float v_scale, double sm_scale, float o_scale,
-                         double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16) {
+void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
+                             int num_q_heads, const uint8_t* cache,
+                             int64_t num_blocks, int block_size, int num_kv_heads,
+                             int head_size, const int32_t* block_table,
+                             int max_blocks_per_seq, const int32_t* seq_lens,
+                             const int32_t* qo_indptr, int num_seqs, float k_scale,
+                             float v_scale, double sm_scale, float o_scale,
+                             double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16,
+                             int kv_format) {
   (void)num_blocks;
   (void)num_q_tokens;
-  int64_t full_dim = nvo_full_dim(head_size);
+  int64_t full_dim = kv_row_bytes(kv_format, head_size);
   int group = num_q_heads / num_kv_heads;
   if (sm_scale <= 0.0) sm_scale = 1.0 / sqrt((double)head_size);
 
@@ -329,7 +345,7 @@ void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
       double dot = 0.0;
       for (int d = 0; d < head_size; ++d)
         dot += (double)nvo_bf16_to_f32(qrow[d]) *
-               (row_elem(krow, head_size, d) * (double)k_scale);
+               (kv_elem(kv_format, krow, head_size, d) * (double)k_scale);
       z[n] = sm_scale * dot;
       if (z[n] > m) m = z[n];
     }
@@ -343,7 +359,7 @@ void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
           cache + row_offset(block, 1, h, (int)(n % block_size), num_kv_heads,
                              block_size, full_dim);
       for (int d = 0; d < head_size; ++d)
-        o[d] += w * (row_elem(vrow, head_size, d) * (double)v_scale);
+        o[d] += w * (kv_elem(kv_format, vrow, head_size, d) * (double)v_scale);
     }
     int64_t out_base = (tok * num_q_heads + hq) * (int64_t)head_size;
     for (int d = 0; d < head_size; ++d) {
@@ -360,6 +376,65 @@ void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
   }
   free(row_seq);
   free(row_idx);
+}
+
+/* NVFP4 cache (the format above). */
+void nvo_paged_attention(const uint16_t* q, int64_t num_q_tokens,
+                         int num_q_heads, const uint8_t* cache,
+                         int64_t num_blocks, int block_size, int num_kv_heads,
+                         int head_size, const int32_t* block_table,
+                         int max_blocks_per_seq, const int32_t* seq_lens,
+                         const int32_t* qo_indptr, int num_seqs, float k_scale,
+                         float v_scale, double sm_scale, float o_scale,
+                         double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16) {
+  nvo_paged_attention_fmt(q, num_q_tokens, num_q_heads, cache, num_blocks,
+                          block_size, num_kv_heads, head_size, block_table,
+                          max_blocks_per_seq, seq_lens, qo_indptr, num_seqs,
+                          k_scale, v_scale, sm_scale, o_scale, o_f64, o_fp8,
+                          o_bf16, NVO_KV_NVFP4);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8-E4M3 KV cache (the comparison format)                                 */
+/* ------------------------------------------------------------------------ */
+
+/* [P1] review highlights and risks: the FP8 KV cache is the format NVFP4 is
+ * compared with (TPOT at batch 256). Reading taken: the FP8 cache has the same
+ * HND page layout with head_size-byte rows of E4M3 codes; the writer stores
+ * E4M3_RNE_satfinite(fl32(x / g)) (IEEE fp32 division, g = k_scale or
+ * v_scale) and the attention reads xhat = E4M3(code) * g. */
+int64_t nvo_fp8kv_quantize_append_paged(const uint16_t* k, const uint16_t* v,
+                                        int64_t k_token_stride,
+                                        int64_t v_token_stride,
+                                        int64_t num_tokens, int num_kv_heads,
+                                        int head_size, uint8_t* cache,
+                                        int64_t num_blocks, int block_size,
+                                        const int64_t* slot_mapping,
+                                        float k_scale, float v_scale) {
+  int64_t bad = 0;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_blocks * block_size) {
+      ++bad;
+      continue;
+    }
+    int64_t block = slot / block_size;
+    int off = (int)(slot % block_size);
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint16_t* src = kv == 0 ? k + t * k_token_stride : v + t * v_token_stride;
+      float g = kv == 0 ? k_scale : v_scale;
+      for (int h = 0; h < num_kv_heads; ++h) {
+        uint8_t* row = cache + row_offset(block, kv, h, off, num_kv_heads,
+                                          block_size, head_size);
+        for (int d = 0; d < head_size; ++d) {
+          float x = nvo_bf16_to_f32(src[(int64_t)h * head_size + d]) / g;
+          row[d] = nvo_e4m3_encode((double)x);
+        }
+      }
+    }
+  }
+  return bad;
 }
 
 /* ------------------------------------------------------------------------ */

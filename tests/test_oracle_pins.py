@@ -426,3 +426,58 @@ def test_activation_rows_are_the_kv_row_codec():
     # g is the inverse of inv, not inv: the scales would change with inv itself
     alt = oracle.quantize_row(np.ascontiguousarray(x[0]), inv)
     assert not np.array_equal(sf[0], alt[cols // 2:])
+
+
+# ------------------------------------------------------------- FP8 KV cache
+def test_fp8kv_writer_vs_torch_cast():
+    """FP8 rows: E4M3 RNE of fl32(x / g), saturating at 448, checked against
+    torch's float8_e4m3fn cast of the same fp32 quotient (clamped first: torch
+    does not saturate); untouched rows keep their sentinel bytes."""
+    rng = np.random.default_rng(12)
+    T, H, D, bs, NB = 40, 2, 64, 16, 6
+    kf = (rng.standard_normal((T, H, D)) * rng.choice([0.01, 1, 50], (T, H, 1))).astype(np.float32)
+    vf = rng.standard_normal((T, H, D)).astype(np.float32)
+    k, v = _bf16_bits(kf), _bf16_bits(vf)
+    gk, gv = float(np.float32(0.013)), float(np.float32(0.7))
+    slots = rng.choice(NB * bs, T, replace=False).astype(np.int64)
+    slots[::7] = -1
+    cache = np.full((NB, 2, H, bs, D), 0xC3, np.uint8)
+    oracle.fp8kv_quantize_append_paged(k, v, cache, slots, gk, gv, bs)
+    for x, g, kv in ((k, gk, 0), (v, gv, 1)):
+        xf = torch.from_numpy((x.astype(np.uint32) << 16).view(np.float32))
+        q = (xf / torch.tensor(g, dtype=torch.float32)).clamp(-448, 448)
+        want = q.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        for t in range(T):
+            if slots[t] < 0:
+                continue
+            blk, off = divmod(int(slots[t]), bs)
+            assert np.array_equal(cache[blk, kv, :, off], want[t])
+    live = {divmod(int(s), bs) for s in slots if s >= 0}
+    for blk in range(NB):
+        for off in range(bs):
+            if (blk, off) not in live:
+                assert (cache[blk, :, :, off] == 0xC3).all()
+
+
+def test_fp8kv_attention_vs_dense_softmax():
+    """FP8-row attention: fp64 oracle vs dense softmax(QK^T)V over hand-packed
+    E4M3 rows decoded by torch, with GQA, prefill rows and g != 1."""
+    rng = np.random.default_rng(13)
+    D, bs, Hkv, G = 64, 16, 2, 2
+    seq_lens, q_lens = [37, 100], [3, 1]
+    NB = sum(-(-L // bs) for L in seq_lens) + 2
+    codes = rng.integers(0, 256, (NB, 2, Hkv, bs, D)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C                     # no NaN codes
+    xhat = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    perm = rng.permutation(NB).astype(np.int32)
+    table = np.zeros((2, 7), np.int32)
+    table[0, :3], table[1, :7] = perm[:3], perm[3:10]
+    qf = rng.standard_normal((sum(q_lens), Hkv * G, D)).astype(np.float32) * 0.05
+    qb = _bf16_bits(qf)
+    qd = ((qb.astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+    indptr = np.array([0, 3, 4], np.int32)
+    gk, gv = float(np.float32(0.02)), float(np.float32(1.3))
+    o64, _, _ = oracle.paged_attention(qb, codes, table, np.array(seq_lens, np.int32), indptr,
+                                       gk, gv, 0.0, 1.0, kv_format=oracle.KV_FP8)
+    ref = _dense_attention(qd, xhat, table, seq_lens, q_lens, G, bs, gk, gv, 1 / math.sqrt(D))
+    np.testing.assert_allclose(o64, ref, rtol=1e-11, atol=1e-12)
