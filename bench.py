@@ -3,9 +3,10 @@
 
 Workload: the Qwen3-0.6B-shaped decode batch (16 q / 8 kv heads, head_size
 128, block_size 16, 32 sequences with 512-4096 keys, N(0,1) K/V with 2% of
-(head, channel) pairs x20, random block tables). One step appends each
-sequence's new token (the quantize-append writer, 32 tokens) and runs decode
-attention over every sequence's keys (FP8 output + bf16 dequant).
+(head, channel) pairs x20, random block tables). One step is one launch of
+the fused decode step: it quantizes and appends each sequence's new token (32
+tokens) and runs decode attention over every sequence's keys (FP8 output +
+bf16 dequant).
 
 Timed region: W warm-up steps, then exactly K steps replayed from CUDA graphs,
 bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
@@ -60,7 +61,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--profile", choices=["attention", "append"], default=None,
+    p.add_argument("--profile", choices=["attention", "append", "step", "activation"],
+                   default=None,
                    help="kernel-only mode for profilers: set up, then launch the chosen "
                         "kernel --steps times (no timing, no JSON)")
     p.add_argument("--workload", default=WORKLOAD, help="workload for --profile attention")
@@ -278,6 +280,12 @@ class DecodeState:
         nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
                            self.ws, o_bf16=self.o16, stream=stream, metadata_ready=metadata_ready)
 
+    def step(self, nk, stream=None, metadata_ready=False):
+        """One decode step in one launch: append the new rows, attend."""
+        nk.paged_decode_append(self.q, self.k_new, self.v_new, self.cache, self.bt, self.sl,
+                               self.kvs, self.o8, self.osc, self.ws, o_bf16=self.o16,
+                               stream=stream, metadata_ready=metadata_ready)
+
 
 def build_cache(w, scales, dev):
     """The workload's whole cache, written by the library's writer."""
@@ -413,6 +421,101 @@ def mixed_record(stream, clocks, region, n_prefill=5, n_decode=20):
     return rec
 
 
+def fp8_kv_record(stream, clocks, region, nvfp4_attn_ms, n_calls=500):
+    """The same decode batch (qwen3_0p6b_decode) over an FP8-E4M3 KV cache:
+    the pages' comparison format (NVFP4 vs FP8 KV TPOT). Decode attention
+    calls back to back over rotated cache copies (> 4x L2)."""
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    from nvfp4_quantized_paged_append_b200 import workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.make_workload(WORKLOAD)
+    scales = wl.global_scales(w, dev)
+    cache = nk.alloc_fp8_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+    ks = torch.tensor([scales[0]], dtype=torch.float32, device=dev)
+    vs = torch.tensor([scales[1]], dtype=torch.float32, device=dev)
+    for b in range(w.num_seqs):
+        k, v = wl.seq_kv(w, b, dev)
+        nk.quantize_append_paged(k, v, cache, torch.from_numpy(w.slots_for_seq(b)).to(dev), ks, vs,
+                                 fp8=True)
+    copies = max(2, -(-4 * L2_BYTES // cache.numel()) + 1)
+    caches = [cache] + [cache.clone() for _ in range(copies - 1)]
+    q = wl.queries(w, dev)
+    bt = torch.from_numpy(w.block_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    kvs = torch.tensor([scales[0], scales[1]], dtype=torch.float32, device=dev)
+    osc = torch.tensor([scales[2]], dtype=torch.float32, device=dev)
+    o8 = torch.empty((w.num_seqs, w.num_q_heads, w.head_size), dtype=torch.uint8, device=dev)
+    o16 = torch.empty_like(o8, dtype=torch.bfloat16)
+    ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, dev)
+    it = [0]
+
+    def once(s):
+        nk.paged_attention(q, caches[it[0] % copies], bt, sl, kvs, o8, osc, ws, o_bf16=o16,
+                           stream=s, fp8=True)
+        it[0] += 1
+
+    time_calls(once, 3, stream, warm=5)
+    clocks.mark()
+    ms = time_calls(once, n_calls, stream)
+    clocks.mark()
+    kvb = int(w.seq_lens.astype(np.int64).sum()) * w.num_kv_heads * 2 * w.head_size
+    peak, kind = peaks()
+    gbs = kvb / (ms * 1e-3) / 1e9
+    rec = {"workload": f"{WORKLOAD} over an FP8-E4M3 KV cache",
+           "kernel": "decode_attention_kernel<128,16,fp8>", "calls": n_calls,
+           "kernel_ms": round(ms, 5), "kv_bytes": kvb, "gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": f"{kind} HBM copy",
+           "nvfp4_kernel_ms": round(nvfp4_attn_ms, 5),
+           "fp8_over_nvfp4_time": round(ms / nvfp4_attn_ms, 3),
+           "l2": f"rotated over {copies} cache copies", "clocks": clocks.summary(region)}
+    del caches, cache
+    torch.cuda.empty_cache()
+    return rec
+
+
+def activation_record(stream, clocks, region, n_calls=200):
+    """Activation NVFP4 quantizer with swizzled scales on an 8192 x 4096 bf16
+    activation (a Qwen3-8B-sized hidden state for 8192 tokens), N(0,1) with 2%
+    of channels x20; inputs rotated over 4 copies (256 MiB > L2)."""
+    import torch
+    import nvfp4_quantized_paged_append_b200 as nk
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rows, cols = 8192, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(8)
+    x = torch.randn((rows, cols), generator=g, device=dev, dtype=torch.float32)
+    x[:, torch.randperm(cols, generator=g, device=dev)[: cols // 50]] *= 20.0
+    x = x.to(torch.bfloat16)
+    inv = torch.tensor([6.0 * 448.0 / float(x.float().abs().amax())], dtype=torch.float32,
+                       device=dev)
+    xs = [x.clone() for _ in range(4)]
+    fp4 = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(nk.activation_sf_bytes(rows, cols, True), dtype=torch.uint8, device=dev)
+    it = [0]
+
+    def once(s):
+        nk.quantize_activation(xs[it[0] % 4], inv, True, fp4, sf, stream=s)
+        it[0] += 1
+
+    time_calls(once, 3, stream, warm=3)
+    clocks.mark()
+    ms = time_calls(once, n_calls, stream)
+    clocks.mark()
+    nbytes = rows * cols * 2 + rows * cols // 2 + sf.numel()
+    peak, kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    rec = {"workload": "activation 8192 x 4096 bf16 -> NVFP4, swizzled scales",
+           "kernel": "quantize_activation_kernel<true>", "calls": n_calls,
+           "kernel_ms": round(ms, 5), "bytes": nbytes,
+           "mtok_s": round(rows / (ms * 1e-3) / 1e6, 1), "gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": f"{kind} HBM copy",
+           "clocks": clocks.summary(region)}
+    del xs, x, fp4, sf
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import nvfp4_quantized_paged_append_b200 as nk
@@ -442,33 +545,52 @@ def run_ours(args, rank, world, dist):
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
     for st in states:  # eager run of every copy before capture (first calls are eager)
+        st.step(nk, stream)
         st.append(nk, stream)
         st.attend(nk, stream)
     stream.synchronize()
-    # Per buffer copy: one CUDA graph for the whole step (append, then the
-    # attention kernel as its programmatic dependent; the block tables and
-    # lengths are step inputs the append does not write, so the attention
-    # kernel reads them while the append finishes) and one for the attention
-    # kernel alone (its own duration, timed back to back).
-    g_step, g_att = [], []
+    # Per buffer copy: one CUDA graph for the step (the fused append + decode
+    # attention kernel, launched as a programmatic dependent of the previous
+    # step's kernel; its block tables and lengths are step inputs no kernel
+    # writes, so it reads them while that kernel finishes), one for the same
+    # step as two kernels (writer, then attention) and one for the attention
+    # kernel alone.
+    g_step, g_two, g_att = [], [], []
+    # one round of steps (one per buffer copy) in one graph: each step's kernel is
+    # a programmatic dependent of the one before, so it starts reading its own
+    # metadata while that kernel finishes (it reads q and the cache only after
+    # that kernel has completed)
+    g_round = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_round, stream=stream):
+        for st in states:
+            st.step(nk, stream, metadata_ready=True)
     for st in states:
         ga = torch.cuda.CUDAGraph()
         with torch.cuda.graph(ga, stream=stream):
+            st.step(nk, stream, metadata_ready=True)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
             st.append(nk, stream)
             st.attend(nk, stream, metadata_ready=True)
         gb = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gb, stream=stream):
             st.attend(nk, stream)
         g_step.append(ga)
+        g_two.append(g2)
         g_att.append(gb)
 
     def run_steps(n):
+        for _ in range(n // copies):
+            g_round.replay()
+        for j in range(n % copies):
+            g_step[j].replay()
+
+    def run_graphs(graphs, n):
         for j in range(n):
-            g_step[j % copies].replay()
+            graphs[j % copies].replay()
 
     def run_attention(n):
-        for j in range(n):
-            g_att[j % copies].replay()
+        run_graphs(g_att, n)
 
     run_steps(max(3, args.warmup))
     stream.synchronize()
@@ -505,6 +627,20 @@ def run_ours(args, rank, world, dist):
     a1.record(stream)
     stream.synchronize()
     attn_ms = a0.elapsed_time(a1) / args.steps
+    # one graph per step (no overlap between consecutive steps), for comparison
+    run_graphs(g_step, max(3, args.warmup))
+    a0.record(stream)
+    run_graphs(g_step, args.steps)
+    a1.record(stream)
+    stream.synchronize()
+    single_ms = a0.elapsed_time(a1) / args.steps
+    # the same step as two kernels (writer, then attention), for comparison
+    run_graphs(g_two, max(3, args.warmup))
+    a0.record(stream)
+    run_graphs(g_two, args.steps)
+    a1.record(stream)
+    stream.synchronize()
+    two_ms = a0.elapsed_time(a1) / args.steps
 
     # ---- quantize-append sweep (8192 tokens) for Mtok/s
     app = wl.make_append()
@@ -548,24 +684,30 @@ def run_ours(args, rank, world, dist):
             x0.record(stream)
         stt = states[it_ % copies]
         stt.stage.copy_(host_stage, non_blocking=True)
-        stt.append(nk, stream)
-        stt.attend(nk, stream)
+        stt.step(nk, stream)
         host_out.copy_(stt.o16, non_blocking=True)
     x1 = torch.cuda.Event(enable_timing=True)
     x1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(x0.elapsed_time(x1) / e2e_steps, dist)
-    del g_step, g_att, states
+    del g_round, g_step, g_two, g_att, states
     torch.cuda.empty_cache()
 
     # ---- the other configurations' kernels: long-context decode and the
     # mixed chunked-prefill batch
     long_rec = long_decode_record(stream, clocks, 1)
     mixed_rec = mixed_record(stream, clocks, 2)
+    act_rec = activation_record(stream, clocks, 3)
+    fp8_rec = fp8_kv_record(stream, clocks, 4, attn_ms)
     clocks.stop()
 
     peak, peak_kind = peaks()
-    achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
+    # the step is one kernel (fused append + decode attention): its duration is
+    # the step time; algorithmic bytes = the KV rows read + the new bf16 rows
+    # read + the new NVFP4 rows written
+    new_rows = w.num_seqs * w.num_kv_heads * 2 * (2 * w.head_size + w.full_dim)
+    step_bytes = kv_bytes + new_rows
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
     traffic = profiled_traffic("decode_attention_kernel<128,16>", WORKLOAD)
     result = {
         "metric": METRIC,
@@ -587,15 +729,21 @@ def run_ours(args, rank, world, dist):
             "kv_bytes_per_step": kv_bytes, "new_tokens_per_step": w.num_seqs,
             "l2": f"inputs rotated over {copies} copies ({copies * cache_bytes / 2**20:.0f} MiB of cache) > 4x L2",
             "parallelism": f"replicas x{world} (independent shards, no collective)",
-            "step": "quantize-append of 32 new tokens + decode attention (one CUDA graph per step)",
+            "step": "one launch: quantize-append of the 32 new tokens fused into decode "
+                    "attention (nvfp4_paged_decode_append); graphs of one step per buffer "
+                    "copy, each launch a programmatic dependent of the previous",
         },
         "roofline": {
-            "bound": "hbm", "kernel": "decode_attention_kernel<128,16>",
+            "bound": "hbm", "kernel": "decode_attention_kernel<128,16> (fused append)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} HBM copy",
-            "traffic": traffic, "algorithmic_bytes_per_launch": kv_bytes,
-            "kernel_ms": round(attn_ms, 5),
+            "traffic": traffic, "algorithmic_bytes_per_launch": step_bytes,
+            "kernel_ms": round(ms_step, 6),
             "frac_of_8TBps": round(achieved / 8000.0, 4),
+            "attention_only_ms": round(attn_ms, 6),
+            "attention_only_frac": round(kv_bytes / (attn_ms * 1e-3) / 1e9 / peak, 4),
+            "two_kernel_step_ms": round(two_ms, 6),
+            "one_graph_per_step_ms": round(single_ms, 6),
         },
         "append": {
             "workload": "append_sweep", "tokens": app.num_tokens, "live_tokens": app.live_tokens(),
@@ -607,14 +755,16 @@ def run_ours(args, rank, world, dist):
         },
         "long_decode": long_rec,
         "mixed_prefill_decode": mixed_rec,
+        "activation_quant": act_rec,
+        "fp8_kv_decode": fp8_rec,
         "e2e": {
             "value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(e2e_ms, 5),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "copies_per_step": "1 H2D (packed inputs) + 1 D2H",
         },
-        # timed region: append + decode attention per step
-        "gpu_launches": 2 * args.steps,
+        # timed region: one fused append + decode attention launch per step
+        "gpu_launches": args.steps,
         "clocks": clocks.summary(0),
     }
     return result
@@ -770,6 +920,32 @@ def run_profile(args):
     import nvfp4_quantized_paged_append_b200 as nk
     from nvfp4_quantized_paged_append_b200 import workloads as wl
     dev = torch.device("cuda", 0)
+    if args.profile == "step":
+        w = wl.make_workload(WORKLOAD)
+        scales = wl.global_scales(w, dev)
+        hist = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
+        ks = torch.tensor([scales[0]], device=dev)
+        vs = torch.tensor([scales[1]], device=dev)
+        for b in range(w.num_seqs):
+            L = int(w.seq_lens[b])
+            k, v = wl.seq_kv(w, b, dev, stop=L - 1)
+            nk.quantize_append_paged(k, v, hist,
+                                     torch.from_numpy(w.slots_for_seq(b, 0, L - 1)).to(dev), ks, vs)
+        st = DecodeState(w, scales, hist, dev)
+        for _ in range(args.steps):
+            st.step(nk)
+        torch.cuda.synchronize()
+        print(f"profile mode: step x{args.steps} done", flush=True)
+        return
+    if args.profile == "activation":
+        rows, cols = 8192, 4096
+        x = torch.randn((rows, cols), device=dev).to(torch.bfloat16)
+        inv = torch.tensor([6.0 * 448.0 / float(x.float().abs().amax())], device=dev)
+        for _ in range(args.steps):
+            nk.quantize_activation(x, inv, True)
+        torch.cuda.synchronize()
+        print(f"profile mode: activation x{args.steps} done", flush=True)
+        return
     if args.profile == "append":
         app = wl.make_append()
         k, v = app.kv(dev)

@@ -184,6 +184,36 @@ NVFP4KV_API int nvfp4_paged_attention_ex(
     void* o_bf16, float* o_f32, void* workspace, size_t workspace_bytes, uint32_t flags,
     nvfp4_stream_t stream);
 
+/* Decode step with the append fused in: one launch that quantizes and writes
+ * every sequence's newest K and V rows into the cache and runs decode
+ * attention over all of each sequence's keys, the new ones included
+ * ("FlashInfer backend adds end-to-end NVFP4 KV cache support", key source
+ * snippets: the forward pass calls reshape_and_cache_flash with the nvfp4
+ * dtype and then the attention kernel; here they are one kernel).
+ * Results equal those of nvfp4_quantize_append_paged (same bytes) followed by
+ * nvfp4_paged_attention on the same stream, with:
+ *   q               bf16 [num_seqs][num_q_heads][head_size] (token b = the
+ *                   query of sequence b), token stride q_token_stride.
+ *   k_new, v_new    bf16 [num_seqs][num_kv_heads][head_size], token strides
+ *                   in elements, 16-byte aligned rows: the newest token of
+ *                   sequence b, written to position seq_lens[b] - 1, i.e. slot
+ *                   block_table[b][(L-1)/block_size]*block_size +
+ *                   (L-1)%block_size with L = seq_lens[b] (>= 1).
+ *   kv_scales       {k_scale, v_scale}: the global scales of the writer and of
+ *                   the attention.
+ * Every other argument, the workspace contract and `flags` are those of
+ * nvfp4_paged_attention_ex (no query ranges: decode only). A new row whose
+ * block id is out of range is neither written nor attended to
+ * (NVFP4_DEV_BAD_BLOCK). */
+NVFP4KV_API int nvfp4_paged_decode_append(
+    const void* q, int64_t q_token_stride, int32_t num_q_heads, const void* k_new,
+    const void* v_new, int64_t k_token_stride, int64_t v_token_stride, uint8_t* cache,
+    int64_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+    const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+    int32_t num_seqs, const float* kv_scales, float sm_scale, uint8_t* o_fp8,
+    const float* o_scale, void* o_bf16, float* o_f32, void* workspace, size_t workspace_bytes,
+    uint32_t flags, nvfp4_stream_t stream);
+
 /* Dequantize listed cache blocks to bf16 ("FlashInfer NVFP4 KV serving on
  * pre-SM100 GPUs", quick answer: the paged NVFP4 dequantize helper).
  *   block_ids       int32 [num_block_ids]: cache blocks to expand.
@@ -195,6 +225,54 @@ NVFP4KV_API int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
                            int32_t num_kv_heads, int32_t head_size,
                            const int32_t* block_ids, int64_t num_block_ids,
                            const float* kv_scales, void* out_bf16, nvfp4_stream_t stream);
+
+/* FP8-E4M3 KV cache: the comparison format of "FlashInfer backend adds
+ * end-to-end NVFP4 KV cache support", review highlights (TPOT of NVFP4 versus
+ * FP8 KV at batch 256). Same HND page layout with head_size-byte rows of E4M3
+ * codes (one per element, no block scales).
+ * nvfp4_fp8kv_quantize_append_paged: arguments, slot rules, status bits and
+ * errors of nvfp4_quantize_append_paged; each element is stored as
+ * E4M3 RNE satfinite(fl32(x / g)), g = *k_scale or *v_scale.
+ * nvfp4_fp8kv_paged_attention: arguments, workspace (the same
+ * nvfp4_paged_attention_workspace_size), flags, outputs and errors of
+ * nvfp4_paged_attention_ex, reading the FP8 cache with xhat = E4M3(code) * g. */
+NVFP4KV_API int nvfp4_fp8kv_quantize_append_paged(
+    const void* k, const void* v, int64_t k_token_stride, int64_t v_token_stride,
+    int64_t num_tokens, int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
+    int64_t num_blocks, int32_t block_size, const int64_t* slot_mapping, const float* k_scale,
+    const float* v_scale, uint32_t* device_status, nvfp4_stream_t stream);
+NVFP4KV_API int nvfp4_fp8kv_paged_attention(
+    const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
+    const uint8_t* cache, int64_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+    int32_t head_size, const int32_t* block_table, int32_t max_blocks_per_seq,
+    const int32_t* seq_lens, const int32_t* qo_indptr, int32_t num_seqs, int32_t max_q_len,
+    const float* kv_scales, float sm_scale, uint8_t* o_fp8, const float* o_scale,
+    void* o_bf16, float* o_f32, void* workspace, size_t workspace_bytes, uint32_t flags,
+    nvfp4_stream_t stream);
+
+/* Activation quantizer for NVFP4 GEMMs ("Move NVFP4 GEMM management into
+ * NvFp4LinearKernel", flashinfer.py and the CUTLASS linear kernel:
+ * scaled_fp4_quant(x, input_global_scale_inv, is_sf_swizzled_layout=True),
+ * swizzle_blockscale). Same group codec as the KV cache rows with the global
+ * scale g = fl32(1 / *global_scale_inv).
+ *   x               bf16 [rows][cols] with row stride row_stride (elements,
+ *                   a multiple of 8, >= cols), 16-byte aligned; cols % 16 == 0.
+ *   global_scale_inv device fp32 scalar (finite, > 0).
+ *   out_fp4         uint8 [rows][cols/2]: E2M1 pairs, element 2j in the low
+ *                   nibble of byte j; 8-byte aligned.
+ *   out_sf          E4M3 scales, nvfp4_activation_sf_bytes(rows, cols,
+ *                   swizzled) bytes. swizzled == 0: [rows][cols/16]. Else rows
+ *                   padded to a multiple of 128 and scale columns to a multiple
+ *                   of 4, 512-byte tiles of 128 rows x 4 scale columns, tile
+ *                   (r/128, c/4) at ((r/128)*(padded columns/4) + c/4)*512,
+ *                   scale (r, c) inside it at (r%32)*16 + ((r%128)/32)*4 + c%4;
+ *                   padding bytes are written as 0.
+ * rows == 0 is a no-op returning NVFP4_OK. */
+NVFP4KV_API size_t nvfp4_activation_sf_bytes(int64_t rows, int64_t cols, int swizzled);
+NVFP4KV_API int nvfp4_quantize_activation(const void* x, int64_t rows, int64_t cols,
+                                          int64_t row_stride, const float* global_scale_inv,
+                                          uint8_t* out_fp4, uint8_t* out_sf, int swizzled,
+                                          nvfp4_stream_t stream);
 
 /* Paged attention that allocates nothing and takes no workspace. The pages
  * this library follows have no counterpart: it exists for callers that

@@ -77,6 +77,18 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_paged_attention_noalloc.argtypes = [P, i64, i64, i32, P, i64, i32, i32, i32, P,
                                                 i32, P, P, i32, i32, P, f32, P, P, P, P, P]
     L.nvfp4_paged_attention_noalloc.restype = ctypes.c_int
+    L.nvfp4_fp8kv_quantize_append_paged.argtypes = L.nvfp4_quantize_append_paged.argtypes
+    L.nvfp4_fp8kv_quantize_append_paged.restype = ctypes.c_int
+    L.nvfp4_fp8kv_paged_attention.argtypes = L.nvfp4_paged_attention_ex.argtypes
+    L.nvfp4_fp8kv_paged_attention.restype = ctypes.c_int
+    L.nvfp4_paged_decode_append.argtypes = [P, i64, i32, P, P, i64, i64, P, i64, i32, i32, i32,
+                                            P, i32, P, i32, P, f32, P, P, P, P, P, sz,
+                                            ctypes.c_uint32, P]
+    L.nvfp4_paged_decode_append.restype = ctypes.c_int
+    L.nvfp4_activation_sf_bytes.argtypes = [i64, i64, ctypes.c_int]
+    L.nvfp4_activation_sf_bytes.restype = sz
+    L.nvfp4_quantize_activation.argtypes = [P, i64, i64, i64, P, P, P, ctypes.c_int, P]
+    L.nvfp4_quantize_activation.restype = ctypes.c_int
     L.nvfp4_dequantize_paged.argtypes = [P, i64, i32, i32, i32, P, i64, P, P, P]
     L.nvfp4_dequantize_paged.restype = ctypes.c_int
     L.nvfp4_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
@@ -127,31 +139,41 @@ def alloc_kv_cache(num_blocks: int, block_size: int, num_kv_heads: int, head_siz
                        dtype=torch.uint8, device=device)
 
 
-def _cache_dims(cache: torch.Tensor):
+def _cache_dims(cache: torch.Tensor, fp8: bool = False):
     if cache.dtype != torch.uint8 or cache.dim() != 5 or cache.shape[1] != 2 or not cache.is_contiguous():
-        raise ValueError("cache must be a contiguous uint8 HND tensor (NB, 2, Hkv, bs, full_dim)")
+        raise ValueError("cache must be a contiguous uint8 HND tensor (NB, 2, Hkv, bs, row bytes)")
     nb, _, hkv, bs, f = cache.shape
+    if fp8:
+        return nb, hkv, bs, f
     d = f * 16 // 9
     if full_dim(d) != f:
         raise ValueError(f"cache last dim {f} is not a valid full_dim")
     return nb, hkv, bs, d
 
 
+def alloc_fp8_kv_cache(num_blocks: int, block_size: int, num_kv_heads: int, head_size: int,
+                       device="cuda") -> torch.Tensor:
+    """uint8 FP8-E4M3 cache in HND order: (num_blocks, 2, num_kv_heads, block_size, head_size)."""
+    return torch.zeros((num_blocks, 2, num_kv_heads, block_size, head_size), dtype=torch.uint8,
+                       device=device)
+
+
 def quantize_append_paged(k: torch.Tensor, v: torch.Tensor, cache: torch.Tensor,
                           slot_mapping: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
                           device_status: Optional[torch.Tensor] = None,
-                          stream: Optional[torch.cuda.Stream] = None) -> None:
-    """Quantize bf16 k/v [T, Hkv, D] into the NVFP4 HND cache at slot_mapping."""
-    nb, hkv, bs, d = _cache_dims(cache)
+                          stream: Optional[torch.cuda.Stream] = None, fp8: bool = False) -> None:
+    """Quantize bf16 k/v [T, Hkv, D] into the NVFP4 HND cache at slot_mapping
+    (fp8=True: into an FP8-E4M3 cache of head_size-byte rows)."""
+    nb, hkv, bs, d = _cache_dims(cache, fp8)
     T = slot_mapping.shape[0]
     for name, x in (("k", k), ("v", v)):
         if x.dtype != torch.bfloat16 or x.shape != (T, hkv, d) or x.stride(2) != 1 or x.stride(1) != d:
             raise ValueError(f"{name} must be bf16 [T, {hkv}, {d}] with contiguous heads")
     if slot_mapping.dtype != torch.int64:
         raise ValueError("slot_mapping must be int64")
-    st = lib().nvfp4_quantize_append_paged(
-        _ptr(k), _ptr(v), k.stride(0), v.stride(0), T, hkv, d, _ptr(cache), nb, bs,
-        _ptr(slot_mapping), _ptr(k_scale), _ptr(v_scale), _ptr(device_status), _stream(stream))
+    fn = lib().nvfp4_fp8kv_quantize_append_paged if fp8 else lib().nvfp4_quantize_append_paged
+    st = fn(_ptr(k), _ptr(v), k.stride(0), v.stride(0), T, hkv, d, _ptr(cache), nb, bs,
+            _ptr(slot_mapping), _ptr(k_scale), _ptr(v_scale), _ptr(device_status), _stream(stream))
     _check(st, "nvfp4_quantize_append_paged")
 
 
@@ -204,10 +226,10 @@ def wait_timeout_probe(status_word: torch.Tensor, polls: int = 1000,
            "nvfp4_wait_timeout_probe")
 
 
-def _attention_dims(q, cache, block_table, seq_lens, qo_indptr, o_fp8, o_bf16, o_f32):
+def _attention_dims(q, cache, block_table, seq_lens, qo_indptr, o_fp8, o_bf16, o_f32, fp8=False):
     """Shape and dtype checks shared by the attention calls; returns
     (num_blocks, Hkv, block_size, D, Tq, Hq, num_seqs, max_blocks_per_seq)."""
-    nb, hkv, bs, d = _cache_dims(cache)
+    nb, hkv, bs, d = _cache_dims(cache, fp8)
     tq, hq, dq = q.shape
     if q.dtype != torch.bfloat16 or dq != d or q.stride(2) != 1 or q.stride(1) != d:
         raise ValueError("q must be bf16 [Tq, Hq, D] with contiguous heads")
@@ -230,21 +252,51 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                     sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
                     o_f32: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None,
-                    metadata_ready: bool = False) -> None:
+                    metadata_ready: bool = False, fp8: bool = False) -> None:
     """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
     metadata_ready: the kernel launched just before on the stream writes none of
     block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
     attention kernel may read them while that kernel finishes
-    (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it)."""
+    (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it).
+    fp8: the cache holds FP8-E4M3 rows (nvfp4_fp8kv_paged_attention)."""
     nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, qo_indptr,
-                                                    o_fp8, o_bf16, o_f32)
-    st = lib().nvfp4_paged_attention_ex(
+                                                    o_fp8, o_bf16, o_f32, fp8)
+    fn = lib().nvfp4_fp8kv_paged_attention if fp8 else lib().nvfp4_paged_attention_ex
+    st = fn(
         _ptr(q), q.stride(0), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
         _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(),
         NVFP4_ATTN_METADATA_READY if metadata_ready else 0, _stream(stream))
     _check(st, "nvfp4_paged_attention")
+
+
+def paged_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                        cache: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                        kv_scales: torch.Tensor, o_fp8: torch.Tensor, o_scale: torch.Tensor,
+                        workspace: torch.Tensor, sm_scale: float = 0.0,
+                        o_bf16: Optional[torch.Tensor] = None,
+                        o_f32: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None,
+                        metadata_ready: bool = False) -> None:
+    """One decode step in one launch: write every sequence's newest k/v row
+    (position seq_lens[b] - 1) into the NVFP4 cache and run decode attention
+    over all keys. q [B, Hq, D], k_new / v_new [B, Hkv, D] bf16."""
+    nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, None,
+                                                    o_fp8, o_bf16, o_f32)
+    for name, x in (("k_new", k_new), ("v_new", v_new)):
+        if x.dtype != torch.bfloat16 or x.shape != (B, hkv, d) or x.stride(2) != 1 or \
+                x.stride(1) != d:
+            raise ValueError(f"{name} must be bf16 [{B}, {hkv}, {d}] with contiguous heads")
+    if tq != B:
+        raise ValueError("q must hold one token per sequence")
+    st = lib().nvfp4_paged_decode_append(
+        _ptr(q), q.stride(0), hq, _ptr(k_new), _ptr(v_new), k_new.stride(0), v_new.stride(0),
+        _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb, _ptr(seq_lens), B, _ptr(kv_scales),
+        float(sm_scale), _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
+        workspace.numel() * workspace.element_size(),
+        NVFP4_ATTN_METADATA_READY if metadata_ready else 0, _stream(stream))
+    _check(st, "nvfp4_paged_decode_append")
 
 
 def paged_attention_noalloc(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
@@ -281,3 +333,34 @@ def dequantize_paged(cache: torch.Tensor, block_ids: torch.Tensor, kv_scales: to
                                       _ptr(kv_scales), _ptr(out), _stream(stream))
     _check(st, "nvfp4_dequantize_paged")
     return out
+
+
+def activation_sf_bytes(rows: int, cols: int, swizzled: bool = True) -> int:
+    return int(lib().nvfp4_activation_sf_bytes(rows, cols, int(swizzled)))
+
+
+def quantize_activation(x: torch.Tensor, global_scale_inv: torch.Tensor, swizzled: bool = True,
+                        out_fp4: Optional[torch.Tensor] = None,
+                        out_sf: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None):
+    """bf16 x [rows, cols] -> (packed E2M1 uint8 [rows, cols/2], E4M3 scales:
+    a flat swizzled uint8 array, or [rows, cols/16] when swizzled is False)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be bf16 [rows, cols] with contiguous rows")
+    rows, cols = x.shape
+    if out_fp4 is None:
+        out_fp4 = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    n = activation_sf_bytes(rows, cols, swizzled)
+    if out_sf is None:
+        out_sf = torch.empty(n, dtype=torch.uint8, device=x.device)
+    if out_fp4.dtype != torch.uint8 or out_fp4.shape != (rows, cols // 2) or \
+            not out_fp4.is_contiguous():
+        raise ValueError("out_fp4 must be contiguous uint8 [rows, cols/2]")
+    if out_sf.dtype != torch.uint8 or out_sf.numel() < n or not out_sf.is_contiguous():
+        raise ValueError(f"out_sf must be contiguous uint8 with >= {n} bytes")
+    st = lib().nvfp4_quantize_activation(_ptr(x), rows, cols, x.stride(0), _ptr(global_scale_inv),
+                                         _ptr(out_fp4), _ptr(out_sf), int(swizzled),
+                                         _stream(stream))
+    _check(st, "nvfp4_quantize_activation")
+    return out_fp4, (out_sf if swizzled else out_sf[:n].view(rows, cols // 16))
+

@@ -111,7 +111,8 @@ int check_attention(const AttentionArgs& a, bool* nothing_to_do) {
   if ((int64_t)a.num_seqs * a.max_blocks_per_seq * a.num_kv_heads >= (int64_t)1 << 30 ||
       a.num_blocks * 2 * a.num_kv_heads >= (int64_t)1 << 31)
     return NVFP4_ERR_UNSUPPORTED;
-  if (decode_warps(a.head_size, a.block_size, a.num_seqs, G) < 1) return NVFP4_ERR_UNSUPPORTED;
+  if (decode_warps(a.head_size, a.block_size, a.num_seqs, G, a.kv_format) < 1)
+    return NVFP4_ERR_UNSUPPORTED;
   return NVFP4_OK;
 }
 
@@ -156,13 +157,12 @@ const char* nvfp4_status_string(int status) {
   }
 }
 
-int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_stride,
-                                int64_t v_token_stride, int64_t num_tokens,
-                                int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
-                                int64_t num_blocks, int32_t block_size,
-                                const int64_t* slot_mapping, const float* k_scale,
-                                const float* v_scale, uint32_t* device_status,
-                                nvfp4_stream_t stream) {
+static int quantize_append_fmt(const void* k, const void* v, int64_t k_token_stride,
+                               int64_t v_token_stride, int64_t num_tokens, int32_t num_kv_heads,
+                               int32_t head_size, uint8_t* cache, int64_t num_blocks,
+                               int32_t block_size, const int64_t* slot_mapping,
+                               const float* k_scale, const float* v_scale,
+                               uint32_t* device_status, nvfp4_stream_t stream, int kv_format) {
   if (num_tokens < 0 || num_kv_heads <= 0 || head_size <= 0 || num_blocks <= 0 ||
       block_size <= 0)
     return NVFP4_ERR_INVALID_ARG;
@@ -179,8 +179,32 @@ int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_st
   nvfp4kv::QuantizeAppendArgs a{k,           v,          k_token_stride, v_token_stride,
                                 num_tokens,  num_kv_heads, head_size,    cache,
                                 num_blocks,  block_size, slot_mapping,   k_scale,
-                                v_scale,     device_status};
+                                v_scale,     device_status, kv_format};
   return cuda_status(nvfp4kv::launch_quantize_append(a, (cudaStream_t)stream));
+}
+
+int nvfp4_quantize_append_paged(const void* k, const void* v, int64_t k_token_stride,
+                                int64_t v_token_stride, int64_t num_tokens,
+                                int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
+                                int64_t num_blocks, int32_t block_size,
+                                const int64_t* slot_mapping, const float* k_scale,
+                                const float* v_scale, uint32_t* device_status,
+                                nvfp4_stream_t stream) {
+  return quantize_append_fmt(k, v, k_token_stride, v_token_stride, num_tokens, num_kv_heads,
+                             head_size, cache, num_blocks, block_size, slot_mapping, k_scale,
+                             v_scale, device_status, stream, 0);
+}
+
+int nvfp4_fp8kv_quantize_append_paged(const void* k, const void* v, int64_t k_token_stride,
+                                      int64_t v_token_stride, int64_t num_tokens,
+                                      int32_t num_kv_heads, int32_t head_size, uint8_t* cache,
+                                      int64_t num_blocks, int32_t block_size,
+                                      const int64_t* slot_mapping, const float* k_scale,
+                                      const float* v_scale, uint32_t* device_status,
+                                      nvfp4_stream_t stream) {
+  return quantize_append_fmt(k, v, k_token_stride, v_token_stride, num_tokens, num_kv_heads,
+                             head_size, cache, num_blocks, block_size, slot_mapping, k_scale,
+                             v_scale, device_status, stream, 1);
 }
 
 size_t nvfp4_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
@@ -207,20 +231,22 @@ int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_t
                                   workspace_bytes, 0u, stream);
 }
 
-int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
-                             int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
-                             int32_t block_size, int32_t num_kv_heads, int32_t head_size,
-                             const int32_t* block_table, int32_t max_blocks_per_seq,
-                             const int32_t* seq_lens, const int32_t* qo_indptr,
-                             int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
-                             float sm_scale, uint8_t* o_fp8, const float* o_scale,
-                             void* o_bf16, float* o_f32, void* workspace,
-                             size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
+static int paged_attention_fmt(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                               int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                               int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                               const int32_t* block_table, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, const int32_t* qo_indptr,
+                               int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                               float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                               void* o_bf16, float* o_f32, void* workspace,
+                               size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream,
+                               int kv_format) {
   if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
   nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
       q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
       head_size, block_table, max_blocks_per_seq, seq_lens, qo_indptr, num_seqs, max_q_len,
       kv_scales, sm_scale, o_fp8, o_scale, o_bf16, o_f32);
+  a.kv_format = kv_format;
   bool nothing_to_do = false;
   const int st = nvfp4kv::check_attention(a, &nothing_to_do);
   if (st != NVFP4_OK || nothing_to_do) return st;
@@ -230,6 +256,36 @@ int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_
   a.workspace = workspace;
   a.flags = flags;
   return nvfp4kv::launch_attention(a, (cudaStream_t)stream);
+}
+
+int nvfp4_paged_attention_ex(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                             int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                             int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                             const int32_t* block_table, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, const int32_t* qo_indptr,
+                             int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                             float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                             void* o_bf16, float* o_f32, void* workspace,
+                             size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
+  return paged_attention_fmt(q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks,
+                             block_size, num_kv_heads, head_size, block_table, max_blocks_per_seq,
+                             seq_lens, qo_indptr, num_seqs, max_q_len, kv_scales, sm_scale, o_fp8,
+                             o_scale, o_bf16, o_f32, workspace, workspace_bytes, flags, stream, 0);
+}
+
+int nvfp4_fp8kv_paged_attention(const void* q, int64_t q_token_stride, int64_t num_q_tokens,
+                                int32_t num_q_heads, const uint8_t* cache, int64_t num_blocks,
+                                int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* qo_indptr,
+                                int32_t num_seqs, int32_t max_q_len, const float* kv_scales,
+                                float sm_scale, uint8_t* o_fp8, const float* o_scale,
+                                void* o_bf16, float* o_f32, void* workspace,
+                                size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
+  return paged_attention_fmt(q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks,
+                             block_size, num_kv_heads, head_size, block_table, max_blocks_per_seq,
+                             seq_lens, qo_indptr, num_seqs, max_q_len, kv_scales, sm_scale, o_fp8,
+                             o_scale, o_bf16, o_f32, workspace, workspace_bytes, flags, stream, 1);
 }
 
 int nvfp4_status_from_bits(uint32_t bits) {
@@ -260,6 +316,60 @@ int nvfp4_wait_timeout_probe(uint32_t* status_word, int32_t polls, nvfp4_stream_
   if (!status_word || !aligned(status_word, 4) || polls < 1 || polls > (1 << 24))
     return NVFP4_ERR_INVALID_ARG;
   return cuda_status(nvfp4kv::launch_wait_timeout_probe(status_word, polls, (cudaStream_t)stream));
+}
+
+int nvfp4_paged_decode_append(const void* q, int64_t q_token_stride, int32_t num_q_heads,
+                              const void* k_new, const void* v_new, int64_t k_token_stride,
+                              int64_t v_token_stride, uint8_t* cache, int64_t num_blocks,
+                              int32_t block_size, int32_t num_kv_heads, int32_t head_size,
+                              const int32_t* block_table, int32_t max_blocks_per_seq,
+                              const int32_t* seq_lens, int32_t num_seqs, const float* kv_scales,
+                              float sm_scale, uint8_t* o_fp8, const float* o_scale, void* o_bf16,
+                              float* o_f32, void* workspace, size_t workspace_bytes,
+                              uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
+  nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
+      q, q_token_stride, num_seqs, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
+      head_size, block_table, max_blocks_per_seq, seq_lens, nullptr, num_seqs, 1, kv_scales,
+      sm_scale, o_fp8, o_scale, o_bf16, o_f32);
+  bool nothing_to_do = false;
+  const int st = nvfp4kv::check_attention(a, &nothing_to_do);
+  if (st != NVFP4_OK || nothing_to_do) return st;
+  if (!k_new || !v_new) return NVFP4_ERR_INVALID_ARG;
+  const int64_t row = (int64_t)num_kv_heads * head_size;
+  if (k_token_stride < row || v_token_stride < row || k_token_stride % 8 != 0 ||
+      v_token_stride % 8 != 0 || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return NVFP4_ERR_INVALID_ARG;
+  const size_t need = nvfp4_paged_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                           head_size);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return NVFP4_ERR_WORKSPACE;
+  a.workspace = workspace;
+  a.flags = flags;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_new_stride = k_token_stride;
+  a.v_new_stride = v_token_stride;
+  return nvfp4kv::launch_attention(a, (cudaStream_t)stream);
+}
+
+size_t nvfp4_activation_sf_bytes(int64_t rows, int64_t cols, int swizzled) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) return 0;
+  const int64_t c16 = cols / 16;
+  if (!swizzled) return (size_t)(rows * c16);
+  return (size_t)(((rows + 127) / 128 * 128) * ((c16 + 3) / 4 * 4));
+}
+
+int nvfp4_quantize_activation(const void* x, int64_t rows, int64_t cols, int64_t row_stride,
+                              const float* global_scale_inv, uint8_t* out_fp4, uint8_t* out_sf,
+                              int swizzled, nvfp4_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0 || row_stride < cols || row_stride % 8 != 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (rows == 0) return NVFP4_OK;
+  if (!x || !global_scale_inv || !out_fp4 || !out_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out_fp4, 8)) return NVFP4_ERR_INVALID_ARG;
+  nvfp4kv::ActivationArgs a{x, rows, cols, row_stride, global_scale_inv, out_fp4, out_sf,
+                            swizzled != 0};
+  return cuda_status(nvfp4kv::launch_quantize_activation(a, (cudaStream_t)stream));
 }
 
 int nvfp4_dequantize_paged(const uint8_t* cache, int64_t num_blocks, int32_t block_size,

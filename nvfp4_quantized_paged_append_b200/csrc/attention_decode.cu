@@ -61,19 +61,25 @@ constexpr size_t kDecodeSmemBudget = 226 * 1024;
 // One persistent CTA per SM: all of an SM's warps belong to the same block, so
 // none of them is starved behind an older co-resident block. head_size 256
 // needs more registers and larger rows: 32-token units and fewer warps.
-template <int D>
+// KV row formats: NVFP4 (E2M1 pairs + E4M3 block scales, D/2 + D/16 bytes)
+// and FP8 (one E4M3 byte per element, D bytes; per-tensor scale only).
+constexpr int kFmtNvfp4 = 0, kFmtFp8 = 1;
+
+template <int D, int FMT = kFmtNvfp4>
 struct DecodeCfg {
-  static constexpr int kUnitTok = (D == 256) ? 32 : 64;
+  // FP8 rows are larger: 32-token units above head_size 64 keep the page rings
+  // of all warps within shared memory
+  static constexpr int kUnitTok = (D == 256 || (FMT == kFmtFp8 && D == 128)) ? 32 : 64;
   static constexpr int kMaxWarps = (D == 256) ? 8 : 12;
   static constexpr int kStages = (D == 64) ? 3 : 2;  // units in flight per warp
 };
 
-template <int D, int BS>
+template <int D, int BS, int FMT = kFmtNvfp4>
 struct DecodeShape {
-  static constexpr int kStages = DecodeCfg<D>::kStages;
-  static constexpr int UT = DecodeCfg<D>::kUnitTok;  // keys per unit
-  static constexpr int T = UT / 16;                   // 16-token tiles per unit
-  static constexpr int F = D / 2 + D / 16;
+  static constexpr int kStages = DecodeCfg<D, FMT>::kStages;
+  static constexpr int UT = DecodeCfg<D, FMT>::kUnitTok;  // keys per unit
+  static constexpr int T = UT / 16;                        // 16-token tiles per unit
+  static constexpr int F = FMT == kFmtFp8 ? D : D / 2 + D / 16;
   static constexpr int PAGE = BS * F;                  // bytes of one (block, K|V, head) page
   static constexpr int U = UT >= BS ? UT / BS : 1;     // pages per unit
   static constexpr int STAGE = 2 * UT * F;             // [K0][V0][K1][V1].. bytes
@@ -98,7 +104,7 @@ struct DecodeShape {
   static int warps_for(int num_seqs, int group) {
     const size_t f = fixed(num_seqs), pw = per_warp(group);
     if (f + pw > kDecodeSmemBudget) return 0;
-    return (int)std::min<size_t>(DecodeCfg<D>::kMaxWarps, (kDecodeSmemBudget - f) / pw);
+    return (int)std::min<size_t>(DecodeCfg<D, FMT>::kMaxWarps, (kDecodeSmemBudget - f) / pw);
   }
   static size_t smem_bytes(int num_seqs, int group, int warps) {
     return warps * per_warp(group) + fixed(num_seqs);
@@ -442,21 +448,133 @@ __device__ __forceinline__ void pv_tile(uint32_t vt, const LaneOffsets& lo, int 
   }
 }
 
+// FP8 rows: per-lane byte offsets inside a 16-token tile. K: lane t4 owns
+// bytes [t4 D/4, (t4+1) D/4) of rows g8 and g8+8 (MMA chunk c uses its word c);
+// V: bytes [g8 D/8, (g8+1) D/8) of tokens 2t4, 2t4+1, 2t4+8, 2t4+9.
+template <int D>
+__device__ __forceinline__ LaneOffsets lane_offsets_fp8(int g8, int t4) {
+  LaneOffsets o;
+  o.k0 = g8 * D + t4 * (D / 4);
+  o.k1 = o.k0 + 8 * D;
+  o.ks0 = o.ks1 = 0;
+  o.va = (2 * t4) * D + g8 * (D / 8);
+  o.vb = o.va + D;
+  o.vc = o.va + 8 * D;
+  o.vd = o.va + 9 * D;
+  o.vsa = o.vsb = o.vsc = o.vsd = 0;
+  return o;
+}
+
+// S^T tile from FP8 rows: E4M3 pairs convert exactly to f16 (no block scale:
+// the per-tensor scale is folded into the logit scale). Rows >= valid are
+// zeroed (stale bytes may hold NaN codes) and get -inf logits (MASK only).
+template <int D, bool MASK>
+__device__ __forceinline__ void qk_tile_fp8(uint32_t kt, const LaneOffsets& lo, int valid, int g8,
+                                            const uint32_t (&bq)[D / 16][2], float (&sacc)[4]) {
+  constexpr int NW = D / 16;  // words per lane and row = MMA chunks
+  uint32_t kw0[NW], kw1[NW];
+#pragma unroll
+  for (int i = 0; i < NW; i += 4) {
+    if constexpr (NW >= 4) {
+      lds_words<16>(kt + lo.k0 + 4 * i, kw0 + i);
+      lds_words<16>(kt + lo.k1 + 4 * i, kw1 + i);
+    }
+  }
+  if constexpr (MASK) {
+    const bool z0 = g8 >= valid, z1 = g8 + 8 >= valid;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      kw0[i] = z0 ? 0u : kw0[i];
+      kw1[i] = z1 ? 0u : kw1[i];
+    }
+  }
+  float s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < NW; ++c) {
+    uint32_t af[4];
+    af[0] = e4m3x2_to_f16x2(kw0[c] & 0xFFFFu);
+    af[1] = e4m3x2_to_f16x2(kw1[c] & 0xFFFFu);
+    af[2] = e4m3x2_to_f16x2(kw0[c] >> 16);
+    af[3] = e4m3x2_to_f16x2(kw1[c] >> 16);
+    if (c & 1) mma_f16_16816(s2, af, bq[c]); else mma_f16_16816(sacc, af, bq[c]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sacc[i] += s2[i];
+  if constexpr (MASK) {
+    if (g8 >= valid) sacc[0] = sacc[1] = -INFINITY;
+    if (g8 + 8 >= valid) sacc[2] = sacc[3] = -INFINITY;
+  }
+}
+
+// O^T += Vhat^T P for one 16-token tile of FP8 rows: A fragments pair the same
+// element of two tokens (byte interleave, then an exact E4M3 -> f16 pair).
+template <int D, bool MASK, bool DUP>
+__device__ __forceinline__ void pv_tile_fp8(uint32_t vt, const LaneOffsets& lo, int valid, int t4,
+                                            const uint32_t (&bp)[2], const uint32_t (&bpl)[2],
+                                            float (&acc)[D / 16][4]) {
+  constexpr int VB = D / 8;  // lane's bytes per token
+  constexpr int VW = VB / 4;
+  uint32_t v0[VW], v1[VW], v2[VW], v3[VW];
+  if constexpr (VB >= 16) {
+#pragma unroll
+    for (int i = 0; i < VW; i += 4) {
+      lds_words<16>(vt + lo.va + 4 * i, v0 + i);
+      lds_words<16>(vt + lo.vb + 4 * i, v1 + i);
+      lds_words<16>(vt + lo.vc + 4 * i, v2 + i);
+      lds_words<16>(vt + lo.vd + 4 * i, v3 + i);
+    }
+  } else {
+    lds_words<8>(vt + lo.va, v0);
+    lds_words<8>(vt + lo.vb, v1);
+    lds_words<8>(vt + lo.vc, v2);
+    lds_words<8>(vt + lo.vd, v3);
+  }
+  if constexpr (MASK) {
+    const bool za = 2 * t4 >= valid, zb = 2 * t4 + 1 >= valid;
+    const bool zc = 2 * t4 + 8 >= valid, zd = 2 * t4 + 9 >= valid;
+#pragma unroll
+    for (int j = 0; j < VW; ++j) {
+      v0[j] = za ? 0u : v0[j];
+      v1[j] = zb ? 0u : v1[j];
+      v2[j] = zc ? 0u : v2[j];
+      v3[j] = zd ? 0u : v3[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < VW; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // chunk m = 2j + h: bytes 2m (even d) and 2m + 1 (odd d)
+      const int m = 2 * j + h;
+      const uint32_t se = h ? 0x0062u : 0x0040u, so = h ? 0x0073u : 0x0051u;
+      uint32_t af[4];
+      af[0] = e4m3x2_to_f16x2(prmt(v0[j], v1[j], se));
+      af[1] = e4m3x2_to_f16x2(prmt(v0[j], v1[j], so));
+      af[2] = e4m3x2_to_f16x2(prmt(v2[j], v3[j], se));
+      af[3] = e4m3x2_to_f16x2(prmt(v2[j], v3[j], so));
+      mma_f16_16816(acc[m], af, bp);
+      if constexpr (!DUP) mma_f16_16816(acc[m], af, bpl);
+    }
+  }
+}
+
 // One unit of T 16-token tiles in the stage at shared address sbase. MASK:
 // tile t holds valid[t] usable keys (0: skipped).
-template <int D, int BS, bool MASK, bool DUP>
+template <int D, int BS, bool MASK, bool DUP, int FMT>
 __device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, const LaneOffsets& lo,
                                             const uint32_t (&bq)[D / 16][2], float qmult,
                                             uint32_t lo_sel, float (&m_run)[2], float (&l_run)[2],
                                             float (&acc)[D / 16][4], int g8, int t4) {
-  using S = DecodeShape<D, BS>;
+  using S = DecodeShape<D, BS, FMT>;
   constexpr int T = S::T, NCH = S::NCH;
   float s[T][4];
 #pragma unroll
   for (int t = 0; t < T; ++t) {
     s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.0f;
     if (!MASK || valid[t] > 0) {
-      qk_tile<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
+      if constexpr (FMT == kFmtFp8)
+        qk_tile_fp8<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
+      else
+        qk_tile<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
     } else {
       s[t][0] = s[t][1] = s[t][2] = s[t][3] = -INFINITY;
     }
@@ -526,8 +644,12 @@ __device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, co
     if (!MASK || valid[t] > 0) {
       uint32_t bp[2], bpl[2];
       p_fragments<DUP>(p[t], lo_sel, bp, bpl);
-      pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp, bpl,
-                            acc);
+      if constexpr (FMT == kFmtFp8)
+        pv_tile_fp8<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp,
+                                  bpl, acc);
+      else
+        pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp,
+                              bpl, acc);
     }
   }
 }
@@ -601,10 +723,10 @@ __device__ __forceinline__ void merge_head(const OutPtrs& op, int num_q_heads,
 
 }  // namespace
 
-template <int D, int BS, bool DUP>
-__global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
+template <int D, int BS, bool DUP, int FMT>
+__global__ void __launch_bounds__(DecodeCfg<D, FMT>::kMaxWarps * 32, 1)
     decode_attention_kernel(const __grid_constant__ AttentionArgs a) {
-  using S = DecodeShape<D, BS>;
+  using S = DecodeShape<D, BS, FMT>;
   constexpr int kStages = S::kStages;
   constexpr int PAGE = S::PAGE, NCH = S::NCH, U = S::U, UT = S::UT, T = S::T;
   constexpr int STAGE = S::STAGE;
@@ -621,9 +743,9 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   int* sub = cum + B + 1;              // [B] units per kv head
   int* slen = sub + B;                 // [B] keys
   int* sqt = slen + B;                 // [B] query token
-  __shared__ int warp_tot[DecodeCfg<D>::kMaxWarps];
-  __shared__ int cut_sg[2 * DecodeCfg<D>::kMaxWarps];  // [warp][slot]: cut segment or -1
-  __shared__ int won[2 * DecodeCfg<D>::kMaxWarps];     // segments this block merges
+  __shared__ int warp_tot[DecodeCfg<D, FMT>::kMaxWarps];
+  __shared__ int cut_sg[2 * DecodeCfg<D, FMT>::kMaxWarps];  // [warp][slot]: cut segment or -1
+  __shared__ int won[2 * DecodeCfg<D, FMT>::kMaxWarps];     // segments this block merges
   __shared__ int nwon;
 
   // Launched as a programmatic dependent of the previous kernel on the stream
@@ -632,6 +754,10 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   // visible. With metadata_ready the batch metadata (sequence lengths, query
   // ranges, block table) is known not to be among them and is read first.
   const bool metadata_ready = (a.flags & kAttnMetadataReady) != 0;
+  // The next kernel on the stream, if launched as a programmatic dependent,
+  // may start its blocks on SMs this grid frees; like this one, it waits for
+  // this grid's completion before reading anything this grid writes.
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   if (!metadata_ready) grid_dependency_wait();
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
@@ -640,7 +766,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
   int* counters = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.counters_off);
   float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.partials_off);
   float* part_ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + wl.ml_off);
-  if (tid < 2 * DecodeCfg<D>::kMaxWarps) cut_sg[tid] = -1;
+  if (tid < 2 * DecodeCfg<D, FMT>::kMaxWarps) cut_sg[tid] = -1;
   if (tid == 0) nwon = 0;
 
   // ---- 1. unit prefix over decode sequences (q_len == 1): a sequence has
@@ -766,11 +892,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
               ids[j] = x;
               ok |= 1 << j;
             } else {
-              atomicOr(status, kDevBadBlock);  // skipped below: a copy of block 0, masked
+              atomicOr(status, kDevBadBlock);  // not copied; its tiles are masked
             }
           }
         }
-        meta = (hh << 16) | (ok << 8) | npg;
+        meta = (hh << 16) | ok;
       }
       if (bank) {
 #pragma unroll
@@ -789,16 +915,16 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
       int blk[U];
 #pragma unroll
       for (int j = 0; j < U; ++j) blk[j] = __shfl_sync(0xffffffffu, bank ? bid1[j] : bid0[j], src);
-      const int n_pg = meta & 0xFF, n_h = meta >> 16;
+      const int cmask = meta & 0xFF, n_h = meta >> 16;  // pages to copy (bit j: page j)
       // The stage being refilled was last read by this warp's own ld.shared
       // instructions, all complete before the __syncwarp that precedes this
       // call; the copies only write, so no proxy fence is needed here.
       if (lane == 0) {
-        my_ok[st] = (meta >> 8) & 0xFF;
-        mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * n_pg);
+        my_ok[st] = meta & 0xFF;  // copied pages
+        mbar_arrive_expect_tx(&my_bars[st], 2 * PAGE * __popc(cmask));
         uint8_t* dst = my_ring_p + (size_t)st * STAGE;
         // page row r of the cache: (block, K|V, head) = (r / 2Hkv, r / Hkv % 2, r % Hkv)
-        if (S::kGather && n_pg == U) {
+        if (S::kGather && cmask == (1 << U) - 1) {
           const uint32_t d = smem_u32(dst);
           if constexpr (U == 4) {
             tma_gather4(d, &a.kv_pages, blk[0] * 2 * Hkv + n_h, blk[1] * 2 * Hkv + n_h,
@@ -814,7 +940,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         } else {
 #pragma unroll
           for (int j = 0; j < U; ++j) {
-            if (j < n_pg) {
+            if ((cmask >> j) & 1) {
               const uint8_t* kp = a.cache + ((long long)blk[j] * 2 * Hkv + n_h) * PAGE;
               bulk_g2s(dst + j * PAGE, kp, PAGE, &my_bars[st]);
               bulk_g2s(dst + (U + j) * PAGE, kp + (long long)Hkv * PAGE, PAGE, &my_bars[st]);
@@ -836,7 +962,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
     for (int k = 0; k < min(kStages, nk); ++k) issue(k);
 
     const float k_scale = __ldg(a.kv_scales);
-    const LaneOffsets lo = lane_offsets<D>(g8, t4);
+    const LaneOffsets lo = FMT == kFmtFp8 ? lane_offsets_fp8<D>(g8, t4) : lane_offsets<D>(g8, t4);
     // DUP: columns G..2G-1 of the lanes' B fragments carry lo parts
     const bool lo0 = DUP && (2 * t4 >= G) && (2 * t4 < 2 * G);
     const bool lo1 = DUP && (2 * t4 + 1 >= G) && (2 * t4 + 1 < 2 * G);
@@ -854,6 +980,55 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
         const int pe = min(r_hi, seg_end);
         const int L = slen[b];
         const int qt = sqt[b];
+
+        // ---- fused append: the warp holding the segment's last unit quantizes
+        // the sequence's newest K and V rows of head h (position L - 1), writes
+        // them to the cache and, once that unit's pages land, over its own
+        // shared-memory copy of the row (no other warp reads that page). Lanes
+        // [0, D/16) take the K groups of 16 elements, [D/16, D/8) the V groups.
+        constexpr int NGR = D / 16;
+        const bool app = FMT == kFmtNvfp4 && a.k_new != nullptr && pe == seg_end && L >= 1;
+        uint32_t app_c0 = 0u, app_c1 = 0u, app_sb = 0u;
+        int app_unit = -1, app_pg = 0, app_off = 0;
+        if (app && !poisoned) {
+          const int pos = L - 1;
+          const int pg = pos / BS;
+          app_off = pos % BS;
+          app_unit = pg / U;
+          app_pg = pg % U;
+          long long blk = -1;
+          if (pg < a.max_blocks_per_seq) {
+            blk = ldg_early(a.block_table + (long long)b * a.max_blocks_per_seq + pg);
+            if (blk < 0 || blk >= a.num_blocks) blk = -1;  // (flagged by the block-id fetch)
+          }
+          if (lane < 2 * NGR) {
+            const int kv = lane / NGR, j = lane % NGR;
+            const __nv_bfloat16* src =
+                reinterpret_cast<const __nv_bfloat16*>(kv ? a.v_new : a.k_new) +
+                (long long)b * (kv ? a.v_new_stride : a.k_new_stride) + (long long)h * D + j * 16;
+            const uint4 r0 = __ldg(reinterpret_cast<const uint4*>(src));
+            const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              x[2 * i] = __uint_as_float(wv[i] << 16);
+              x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+            }
+            app_sb = quantize_group16(x, __ldg(a.kv_scales + kv), app_c0, app_c1);
+            if (blk >= 0) {
+              uint8_t* dst = const_cast<uint8_t*>(a.cache) +
+                             ((blk * 2 + kv) * Hkv + h) * (long long)PAGE + app_off * S::F;
+              if constexpr (S::F % 8 == 0) {
+                *reinterpret_cast<uint2*>(dst + 8 * j) = make_uint2(app_c0, app_c1);
+              } else {
+                reinterpret_cast<uint32_t*>(dst + 8 * j)[0] = app_c0;
+                reinterpret_cast<uint32_t*>(dst + 8 * j)[1] = app_c1;
+              }
+              dst[D / 2 + j] = (uint8_t)app_sb;
+            }
+          }
+        }
 
         // ---- query fragments from this warp's query buffer: lane (g8, t4)
         // holds q[head of column g8][t4*D/4 + i]. DUP: columns G..2G-1 repeat
@@ -929,9 +1104,28 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
             }
           }
           const uint32_t sbase = my_ring + st * STAGE;
+          if (u == app_unit && ((okbits >> app_pg) & 1)) {
+            // the newest row over this warp's copy of its page (K, then V)
+            if (lane < 2 * NGR) {
+              const int kv = lane / NGR, j = lane % NGR;
+              uint8_t* row = my_ring_p + (size_t)st * STAGE + (kv * U + app_pg) * PAGE +
+                             app_off * S::F;
+              if constexpr (S::F % 8 == 0) {
+                *reinterpret_cast<uint2*>(row + 8 * j) = make_uint2(app_c0, app_c1);
+              } else {
+                reinterpret_cast<uint32_t*>(row + 8 * j)[0] = app_c0;
+                reinterpret_cast<uint32_t*>(row + 8 * j)[1] = app_c1;
+              }
+              row[D / 2 + j] = (uint8_t)app_sb;
+            }
+            // (later bulk copies refill this stage: order these writes first)
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
           const int rem = L - u * UT;  // keys of this unit (clipped per tile below)
-          if (rem >= UT && okbits == (1 << U) - 1) {
-            decode_unit<D, BS, false, DUP>(sbase, nullptr, lo, bq, qmult, lo_sel, m_run, l_run,
+          const int pmask = okbits & 0xFF;  // pages copied
+          if (rem >= UT && pmask == (1 << U) - 1) {
+            decode_unit<D, BS, false, DUP, FMT>(sbase, nullptr, lo, bq, qmult, lo_sel, m_run, l_run,
                                            acc, g8, t4);
           } else {
             int vv[T];
@@ -939,12 +1133,12 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kMaxWarps * 32, 1)
 #pragma unroll
             for (int t = 0; t < T; ++t) {
               int v = min(16, rem - 16 * t);
-              if (v < 0 || !((okbits >> (16 * t / BS)) & 1)) v = 0;
+              if (v < 0 || !((pmask >> (16 * t / BS)) & 1)) v = 0;
               vv[t] = v;
               any |= v > 0;
             }
             if (any)
-              decode_unit<D, BS, true, DUP>(sbase, vv, lo, bq, qmult, lo_sel, m_run, l_run, acc,
+              decode_unit<D, BS, true, DUP, FMT>(sbase, vv, lo, bq, qmult, lo_sel, m_run, l_run, acc,
                                             g8, t4);
           }
           __syncwarp();
@@ -1105,20 +1299,20 @@ static cudaError_t encode_page_rows(CUtensorMap* map, const uint8_t* cache, int6
 // one).
 struct DeviceFacts {
   int sms = 0;
-  unsigned long long ctx[2] = {0, 0};  // context the attribute was set in, per DUP
-  bool smem_attr_set[2] = {false, false};
+  unsigned long long ctx = 0;  // context the attribute was set in
+  bool smem_attr_set = false;
 };
 
-template <int D, int BS, bool DUP>
+template <int D, int BS, bool DUP, int FMT>
 static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) {
-  using S = DecodeShape<D, BS>;
+  using S = DecodeShape<D, BS, FMT>;
   static std::mutex facts_mutex;
   static DeviceFacts facts[64];
   const int G = a.num_q_heads / a.num_kv_heads;
   const int nw = S::warps_for(a.num_seqs, G);
   if (nw < 1) return cudaErrorInvalidValue;
   const size_t smem = S::smem_bytes(a.num_seqs, G, nw);
-  auto kern = decode_attention_kernel<D, BS, DUP>;
+  auto kern = decode_attention_kernel<D, BS, DUP, FMT>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -1130,7 +1324,7 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   {
     std::lock_guard<std::mutex> lock(facts_mutex);
     DeviceFacts& f = facts[dev];
-    if (!f.smem_attr_set[DUP] || ctx == 0 || f.ctx[DUP] != ctx) {
+    if (!f.smem_attr_set || ctx == 0 || f.ctx != ctx) {
       // allow the largest dynamic size the device permits beside the static part
       int optin = 0;
       err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -1143,8 +1337,8 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
       if (err != cudaSuccess) return err;
       err = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev);
       if (err != cudaSuccess) return err;
-      f.smem_attr_set[DUP] = true;
-      f.ctx[DUP] = ctx;
+      f.smem_attr_set = true;
+      f.ctx = ctx;
     }
     sms = f.sms;
   }
@@ -1175,9 +1369,11 @@ static cudaError_t launch_decode_t(const AttentionArgs& a, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
-int decode_warps(int head_size, int block_size, int num_seqs, int group) {
-#define NVFP4_WARPS_CASE(DD, BB) \
-  if (head_size == DD && block_size == BB) return DecodeShape<DD, BB>::warps_for(num_seqs, group);
+int decode_warps(int head_size, int block_size, int num_seqs, int group, int kv_format) {
+#define NVFP4_WARPS_CASE(DD, BB)                                                   \
+  if (head_size == DD && block_size == BB)                                         \
+    return kv_format == kFmtFp8 ? DecodeShape<DD, BB, kFmtFp8>::warps_for(num_seqs, group) \
+                                : DecodeShape<DD, BB, kFmtNvfp4>::warps_for(num_seqs, group);
   NVFP4_WARPS_CASE(64, 16)
   NVFP4_WARPS_CASE(64, 32)
   NVFP4_WARPS_CASE(128, 16)
@@ -1190,10 +1386,15 @@ int decode_warps(int head_size, int block_size, int num_seqs, int group) {
 
 cudaError_t launch_decode_attention(const AttentionArgs& a, cudaStream_t stream) {
   const bool dup = (a.num_q_heads / a.num_kv_heads) <= 4;
-#define NVFP4_DECODE_CASE(DD, BB)                         \
-  if (a.head_size == DD && a.block_size == BB)            \
-    return dup ? launch_decode_t<DD, BB, true>(a, stream) \
-               : launch_decode_t<DD, BB, false>(a, stream);
+  const bool fp8 = a.kv_format == kFmtFp8;
+#define NVFP4_DECODE_CASE(DD, BB)                                                   \
+  if (a.head_size == DD && a.block_size == BB) {                                    \
+    if (fp8)                                                                        \
+      return dup ? launch_decode_t<DD, BB, true, kFmtFp8>(a, stream)                \
+                 : launch_decode_t<DD, BB, false, kFmtFp8>(a, stream);              \
+    return dup ? launch_decode_t<DD, BB, true, kFmtNvfp4>(a, stream)                \
+               : launch_decode_t<DD, BB, false, kFmtNvfp4>(a, stream);              \
+  }
   NVFP4_DECODE_CASE(64, 16)
   NVFP4_DECODE_CASE(64, 32)
   NVFP4_DECODE_CASE(128, 16)

@@ -1,305 +1,593 @@
-// Chunked-prefill attention over the NVFP4 paged cache.
+// Chunked-prefill attention over the NVFP4 paged cache on the Blackwell tensor
+// cores (tcgen05, fp32 accumulators in tensor memory).
 //
 // ("FlashInfer backend adds end-to-end NVFP4 KV cache support",
-// implementation breakdown items 2-3: the prefill wrapper reads the NVFP4
-// pages plus FP8 block scales and writes FP8 output.) Each sequence with
-// q_len > 1 query tokens: query row r sits at position L - q_len + r and
-// attends causally to keys 0..L-q_len+r of its paged cache.
+// implementation breakdown items 2-3: the prefill path reads the NVFP4 pages
+// plus their FP8 block scales and writes FP8 output dequantized back to the
+// model dtype.) Each sequence with q_len > 1 query tokens: query row r sits at
+// position L - q_len + r and attends causally to keys 0..L-q_len+r of its
+// paged cache; o = softmax(sm_scale * q K^T) V with K = E2M1 * E4M3 * k_scale
+// and V likewise with v_scale.
 //
-// CTA = 4 warps x 16 rows; a row is one (query token, query head of the kv
-// head's GQA group) pair, so the 64 rows of a CTA share one kv head and every
-// page is read and dequantized once for all of them. Per page: one bulk async
-// copy each for the K and V page (double-buffered on mbarriers), a
-// cooperative dequant into f16 tiles in shared memory (exact: E2M1 * E4M3 has
-// at most 6 significant bits), then mma.m16n8k16 for S = Q K^T and O += P V
-// with fp32 accumulators and an exp2-domain online softmax.
+// A CTA owns M = 128 rows: 128/G query tokens x the G query heads of one kv
+// head (GQA), so every key chunk is read and dequantized once for all of them.
+// Keys advance in chunks of 64:
+//   S  = Q K^T   tcgen05.mma kind::f16, A = Q (f16, in TMEM), B = K chunk
+//                (f16, 128B-swizzled shared tile, K-major), D = S (fp32, TMEM)
+//   P  = exp2(S * scale - m) in fp32, split into f16 hi + lo (~22 bits: f16
+//        alone misses the 2e-3 bound on outlier-heavy rows), written back to
+//        TMEM over S's columns
+//   O += P V     A = P hi, then P lo (TMEM), B = V chunk (the same swizzled
+//                tile layout read MN-major), D = O (fp32, TMEM)
+// E2M1 * E4M3 has at most 6 significant bits in [2^-10, 2688], so K and V are
+// exact in f16; k_scale is folded into the logit scale and v_scale into the
+// output. Q is scaled per row by a power of two putting max |q| in
+// [2^14, 2^15), where f16 keeps every bf16 bit. The running max moves only when
+// a chunk's max exceeds it by more than 2^8 (then O is rescaled in TMEM).
+//
+// Warp roles (13 warps):
+//   0-3   Q rows into TMEM, softmax (thread i = row i = TMEM lane i), epilogue
+//   4     TMEM allocation; one thread issues every MMA and commit
+//   5-8   K pages: bulk copies of a chunk's NVFP4 pages into a 3-stage ring,
+//         then dequantization into one of two f16 K tiles
+//   9-12  V pages: the same for V
+// Every mbarrier wait is bounded; a wait that gives up raises NVFP4_DEV_TIMEOUT
+// and makes the whole block stop, wait for its copies and MMAs, free its TMEM
+// and return.
 #include <mutex>
 
 #include "nvfp4kv_device.cuh"
 #include "nvfp4kv_launch.h"
+#include "nvfp4kv_tc.cuh"
 
 namespace nvfp4kv {
 
 namespace {
-constexpr int kPWarps = 4;
-constexpr int kRows = kPWarps * 16;
-constexpr float kPLog2e = 1.4426950408889634f;
+constexpr int kRows = 128;   // M of every MMA: (query token, head) rows per CTA
+constexpr int kSBufs = 3;    // S/P buffers in TMEM
+constexpr int kRawStages = 3;
+constexpr int kThreads = 13 * 32;
+constexpr int kMmaWarp = 4;
+constexpr int kKGroup0 = 5 * 32;  // first thread of the K warps
+constexpr int kVGroup0 = 9 * 32;  // first thread of the V warps
+constexpr uint32_t kBarK = 1, kBarV = 2, kBarSoftmax = 3;  // named barriers (128 threads)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThresh = 8.0f;
+constexpr int kMaxPolls = 1 << 22;
+// a CTA keeps the SM to itself (its TMEM allocation is the whole SM's)
+constexpr size_t kMinSmem = 120 * 1024;
 
-template <int D, int BS>
-struct PrefillShape {
-  static constexpr int F = D / 2 + D / 16;
-  static constexpr int PAGE = BS * F;
-  static constexpr int LD = D + 8;  // f16 row stride of the smem tiles (bank spread)
-  static size_t smem_bytes() {
-    return 2ull * 2 * PAGE            // raw K,V pages, two stages
-           + 2ull * kRows * LD        // Q tile (f16)
-           + 2ull * 2 * BS * LD       // dequantized K and V tiles (f16)
-           + 64;                      // mbarriers + scratch
-  }
+// Barrier slots.
+enum : int {
+  kBarKraw = 0,                   // [3] K raw stage filled (expect_tx)
+  kBarVraw = kRawStages,          // [3] V raw stage filled
+  kBarKFull = 2 * kRawStages,     // [2] K tile dequantized (128 arrivals)
+  kBarVFull = kBarKFull + 2,      // [2] V tile dequantized (128 arrivals)
+  kBarKEmpty = kBarVFull + 2,     // [2] S MMAs that read the K tile done (commit)
+  kBarVEmpty = kBarKEmpty + 2,    // [2] PV MMAs that read the V tile done (commit)
+  kBarSFull = kBarVEmpty + 2,     // [3] S chunk in TMEM (commit)
+  kBarPFull = kBarSFull + kSBufs, // [3] P chunk in TMEM (128 arrivals)
+  kBarPFree = kBarPFull + kSBufs, // [3] PV MMAs that read a P buffer done (commit)
+  kBarODone = kBarPFree + kSBufs, // PV MMAs of a chunk done (commit)
+  kBarQReady = kBarODone + 1,     // Q rows in TMEM (128 arrivals)
+  kBarFin = kBarQReady + 1,       // every MMA issued done (commit)
+  kNumBarriers = kBarFin + 1
 };
-}  // namespace
 
-template <int D, int BS>
-__global__ void __launch_bounds__(kPWarps * 32) prefill_attention_kernel(const AttentionArgs a) {
-  using S = PrefillShape<D, BS>;
-  constexpr int F = S::F, PAGE = S::PAGE, LD = S::LD;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* raw = smem;                                              // [2][2][PAGE]
-  __half* Qs = reinterpret_cast<__half*>(raw + 2 * 2 * PAGE);        // [kRows][LD]
-  __half* Ks = Qs + kRows * LD;                                      // [BS][LD]
-  __half* Vs = Ks + BS * LD;                                         // [BS][LD]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + BS * LD);        // [2]
-  float* red = reinterpret_cast<float*>(bars + 2);                   // [4]
-  int* okf = reinterpret_cast<int*>(red + 4);                        // [2]
-
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int g8 = lane >> 2, t4 = lane & 3;
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int Hkv = a.num_kv_heads, G = a.num_q_heads / Hkv;
-  const int tpt = kRows / G;  // query tokens per CTA
-  const int q_begin = a.qo_indptr[b];
-  const int q_len = a.qo_indptr[b + 1] - q_begin;
-  if (q_len <= 1) return;  // decode rows are served by the decode kernel
-  if (q_len > (int)gridDim.x * tpt && blockIdx.x == 0 && threadIdx.x == 0)
-    atomicOr(reinterpret_cast<uint32_t*>(a.workspace), kDevBadQlen);  // rows beyond the grid
-  const int qtok0 = blockIdx.x * tpt;
-  if (qtok0 >= q_len) return;
-  const int L = a.seq_lens[b];
-  const int last_tok = min(q_len - 1, qtok0 + tpt - 1);
-  const int kv_end = min(L, max(0, L - q_len + last_tok + 1));  // keys [0, kv_end) are needed
-  uint32_t* status = reinterpret_cast<uint32_t*>(a.workspace);
-  const float k_scale = __ldg(a.kv_scales), v_scale = __ldg(a.kv_scales + 1);
-  const float o_scale = __ldg(a.o_scale);
-
-  // ---- Q tile -> shared (bf16 first), max |q|, then f16 with a power-of-two scale
-  float mx = 0.0f;
-  for (int c = tid; c < kRows * (D / 8); c += kPWarps * 32) {
-    const int r = c / (D / 8), j = c % (D / 8);
-    const int qt = qtok0 + r / G;
-    uint4 v4 = make_uint4(0, 0, 0, 0);
-    if (r < tpt * G && qt < q_len) {
-      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                 (long long)(q_begin + qt) * a.q_token_stride +
-                                 (long long)(h * G + r % G) * D + 8 * j;
-      v4 = __ldg(reinterpret_cast<const uint4*>(src));
-    }
-    const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      mx = fmaxf(mx, fabsf(__uint_as_float(wv[i] << 16)));
-      mx = fmaxf(mx, fabsf(__uint_as_float(wv[i] & 0xFFFF0000u)));
-    }
-    *reinterpret_cast<uint4*>(Qs + r * LD + 8 * j) = v4;
+template <int D, int BS, int FMT>
+struct PrefillShape {
+  // keys per chunk: N of S = Q K^T and the K-extent of O += P V (32 at head
+  // size 256, where three S/P buffers must fit beside O and Q in TMEM)
+  static constexpr int kChunk = D == 256 ? 32 : 64;
+  static constexpr int F = FMT ? D : D / 2 + D / 16;  // row bytes: NVFP4, or FP8 (FMT = 1)
+  static constexpr int PAGE = BS * F;          // bytes of one (block, K|V, head) page
+  static constexpr int PPC = kChunk >= BS ? kChunk / BS : 1;  // pages per chunk
+  static constexpr int RAW = kChunk * F;       // cache bytes of a chunk (K or V)
+  static constexpr int TILE = kChunk * D * 2;  // f16 tile of a chunk
+  static constexpr int DB = D / 64;            // 64-column blocks of a tile
+  // TMEM columns: O [0, D), S/P buffers [D, D + 3 chunk), Q after them (D/2)
+  static constexpr uint32_t kColO = 0, kColS = D, kColQ = D + kSBufs * kChunk;
+  static constexpr uint32_t kTmemCols = (kColQ + D / 2 <= 256) ? 256u : 512u;
+  // shared memory (offsets from a 1024-aligned base)
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = 2 * TILE;
+  static constexpr int kOffKraw = 4 * TILE;
+  static constexpr int kOffVraw = kOffKraw + kRawStages * RAW;
+  static constexpr int kOffBar = kOffVraw + kRawStages * RAW;
+  static constexpr int kNumBars = kNumBarriers;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kBytes = kOffMisc + 64;
+  static size_t smem_bytes() {
+    const size_t need = (size_t)kBytes + 1024;  // + alignment of the base
+    return need > kMinSmem ? need : kMinSmem;
   }
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[w] = mx;
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_mbar_init();
+  static_assert(RAW % 16 == 0 && PAGE % 16 == 0, "bulk copies move 16-byte multiples");
+  static_assert(TILE % 1024 == 0, "swizzle atoms sit on 1024-byte boundaries");
+  static_assert(kColQ + D / 2 <= 512, "TMEM budget");
+  static_assert(kChunk % BS == 0, "a chunk holds whole pages");
+  static_assert(kOffMisc + 64 <= kBytes, "misc block fits");
+};
+
+struct Misc {
+  uint32_t tmem_base;
+  int abort;  // a wait of some role gave up: everyone stops
+  // per role group (K, V, softmax), two alternating slots: chunk c's stop flag
+  // is written before the group's barrier of chunk c and read after it; the
+  // slot is written again only at chunk c + 2, after every thread of the group
+  // has passed the barrier of chunk c + 1
+  int group_stop[3][2];
+  uint32_t raw_ok[2][kRawStages];  // per raw stage: bit i = page i of the chunk was copied
+};
+
+// Bounded wait that also gives up once another role has aborted the block.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* misc,
+                                         uint32_t* status) {
+  for (int i = 0; i < kMaxPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 127) == 127 && *reinterpret_cast<volatile int*>(&misc->abort)) return false;
   }
-  __syncthreads();
-  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
-  const int sh = min(126, max(-126, 15 - ex));
-  const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
-  const float qmult = a.sm_scale * k_scale * kPLog2e * __uint_as_float((uint32_t)(127 - sh) << 23);
-  for (int c = tid; c < kRows * (D / 8); c += kPWarps * 32) {
-    const int r = c / (D / 8), j = c % (D / 8);
-    uint4* p = reinterpret_cast<uint4*>(Qs + r * LD + 8 * j);
-    uint4 v4 = *p;
-    uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+  atomicOr(status, kDevTimeout);
+  *reinterpret_cast<volatile int*>(&misc->abort) = 1;
+  return false;
+}
+
+// Issue the bulk copies of chunk c's pages (K: kv = 0, V: kv = 1) into raw
+// stage `st`; pages past kv_end or with a bad block id are not copied (the
+// latter flagged). One thread.
+template <int D, int BS, int FMT>
+__device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h, int kv, int c,
+                                            int kv_end, uint8_t* raw, uint64_t* bar,
+                                            uint32_t* ok_out, uint32_t* status) {
+  using S = PrefillShape<D, BS, FMT>;
+  const int Hkv = a.num_kv_heads;
+  uint32_t ok = 0, bytes = 0;
+  long long src[S::PPC];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      wv[i] = pack_f16x2(__uint_as_float(wv[i] << 16) * qs, __uint_as_float(wv[i] & 0xFFFF0000u) * qs);
-    *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-  }
-
-  const int npages = min(a.max_blocks_per_seq, (kv_end + BS - 1) / BS);
-  auto issue = [&](int pg) {  // thread 0 only
-    long long blk = __ldg(a.block_table + (long long)b * a.max_blocks_per_seq + pg);
-    int ok = 1;
-    if (blk < 0 || blk >= a.num_blocks) {
-      atomicOr(status, kDevBadBlock);
-      ok = 0;
-      blk = 0;
-    }
-    const int st = pg & 1;
-    okf[st] = ok;
-    const uint8_t* kp = a.cache + ((blk * 2) * Hkv + h) * (long long)PAGE;
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&bars[st], 2 * PAGE);
-    bulk_g2s(raw + st * 2 * PAGE, kp, PAGE, &bars[st]);
-    bulk_g2s(raw + st * 2 * PAGE + PAGE, kp + (long long)Hkv * PAGE, PAGE, &bars[st]);
-  };
-  if (tid == 0 && npages > 0) issue(0);
-
-  // rows of this lane: warp row base + g8 and + 8
-  const int rA = w * 16 + g8, rB = rA + 8;
-  const int posA = L - q_len + qtok0 + rA / G;  // absolute query positions
-  const int posB = L - q_len + qtok0 + rB / G;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  float acc[D / 8][4];
-#pragma unroll
-  for (int j = 0; j < D / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  bool poisoned = false;
-
-  for (int pg = 0; pg < npages; ++pg) {
-    const int st = pg & 1;
-    if (tid == 0 && pg + 1 < npages && !poisoned) issue(pg + 1);
-    bool ok = false;
-    if (!poisoned) {
-      if (mbar_wait_bounded(&bars[st], (uint32_t)((pg >> 1) & 1))) {
-        ok = okf[st] != 0;
+  for (int i = 0; i < S::PPC; ++i) {
+    const int p = c * S::PPC + i;
+    src[i] = -1;
+    if (p * BS < kv_end && p < a.max_blocks_per_seq) {
+      const long long blk = __ldg(a.block_table + (long long)b * a.max_blocks_per_seq + p);
+      if (blk >= 0 && blk < a.num_blocks) {
+        src[i] = ((blk * 2 + kv) * Hkv + h) * (long long)S::PAGE;
+        ok |= 1u << i;
+        bytes += S::PAGE;
       } else {
-        poisoned = true;
-        if (tid == 0) atomicOr(status, kDevTimeout);
+        atomicOr(status, kDevBadBlock);
       }
     }
-    // ---- dequant K and V pages into f16 tiles (masked rows -> 0)
-    for (int c = tid; c < 2 * BS * (D / 8); c += kPWarps * 32) {
-      const int kv = c / (BS * (D / 8));
-      const int rem = c % (BS * (D / 8));
-      const int r = rem / (D / 8), j = rem % (D / 8);
-      const uint8_t* row = raw + st * 2 * PAGE + kv * PAGE + r * F;
-      const bool valid = ok && (pg * BS + r < kv_end);
-      const uint32_t codes = ld_shared_u32(smem_u32(row + 4 * j));
-      const uint32_t sb = valid ? row[D / 2 + j / 2] : 0u;
-      const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
-      uint32_t o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = hmul2_u32(e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu), s2);
-      __half* dst = (kv == 0 ? Ks : Vs) + r * LD + 8 * j;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    __syncthreads();
-
-#pragma unroll
-    for (int sub = 0; sub < BS / 16; ++sub) {
-      const int key0 = pg * BS + sub * 16;
-      // ---- S = Q K^T (16 rows x 16 keys)
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t af[4], bf[4];
-        const int ar = w * 16 + (lane & 15), acol = c * 16 + (lane >> 4) * 8;
-        ldmatrix_x4(af, smem_u32(Qs + ar * LD + acol));
-        // matrices: (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
-        const int kr = sub * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int kc = c * 16 + ((lane >> 3) & 1) * 8;
-        ldmatrix_x4(bf, smem_u32(Ks + kr * LD + kc));
-        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-        mma_f16_16816(sc[0], af, b0);
-        mma_f16_16816(sc[1], af, b1);
-      }
-      // ---- mask + online softmax (rows rA: c0,c1; rB: c2,c3)
-      float mxA = -INFINITY, mxB = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-          const int key = key0 + nt * 8 + 2 * t4 + e2;
-          const bool kin = ok && key < kv_end;
-          sc[nt][e2] = (kin && key <= posA) ? sc[nt][e2] * qmult : -INFINITY;
-          sc[nt][2 + e2] = (kin && key <= posB) ? sc[nt][2 + e2] * qmult : -INFINITY;
-          mxA = fmaxf(mxA, sc[nt][e2]);
-          mxB = fmaxf(mxB, sc[nt][2 + e2]);
-        }
-      }
-      mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 1));
-      mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 2));
-      mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 1));
-      mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 2));
-      const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
-      const float muA = (mnA == -INFINITY) ? 0.f : mnA, muB = (mnB == -INFINITY) ? 0.f : mnB;
-      const float alA = ex2(m_run[0] - muA), alB = ex2(m_run[1] - muB);
-      m_run[0] = mnA;
-      m_run[1] = mnB;
-      float pA[4], pB[4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        pA[2 * nt] = ex2(sc[nt][0] - muA);
-        pA[2 * nt + 1] = ex2(sc[nt][1] - muA);
-        pB[2 * nt] = ex2(sc[nt][2] - muB);
-        pB[2 * nt + 1] = ex2(sc[nt][3] - muB);
-      }
-      l_run[0] = l_run[0] * alA + pA[0] + pA[1] + pA[2] + pA[3];
-      l_run[1] = l_run[1] * alB + pB[0] + pB[1] + pB[2] + pB[3];
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        acc[j][0] *= alA;
-        acc[j][1] *= alA;
-        acc[j][2] *= alB;
-        acc[j][3] *= alB;
-      }
-      // P as the A operand: (rA, k 2t4..), (rB, k 2t4..), (rA, k 2t4+8..), (rB, k 2t4+8..),
-      // split into f16 hi + lo parts (hi = f16(p), lo = f16(p - hi)) so P keeps ~22 bits
-      const uint32_t pa[4] = {pack_f16x2(pA[0], pA[1]), pack_f16x2(pB[0], pB[1]),
-                              pack_f16x2(pA[2], pA[3]), pack_f16x2(pB[2], pB[3])};
-      float lA[4], lB[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lA[i] = pA[i] - __half2float(__float2half_rn(pA[i]));
-        lB[i] = pB[i] - __half2float(__float2half_rn(pB[i]));
-      }
-      const uint32_t pl[4] = {pack_f16x2(lA[0], lA[1]), pack_f16x2(lB[0], lB[1]),
-                              pack_f16x2(lA[2], lA[3]), pack_f16x2(lB[2], lB[3])};
-      // ---- O += P V
-#pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        uint32_t bf[4];
-        // matrices: (keys 0-7, d 16j..), (keys 8-15, d 16j..), (keys 0-7, d 16j+8..), (keys 8-15, d 16j+8..)
-        const int vr = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int vc = j * 16 + (lane >> 4) * 8;
-        ldmatrix_x4_trans(bf, smem_u32(Vs + vr * LD + vc));
-        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-        mma_f16_16816(acc[2 * j], pa, b0);
-        mma_f16_16816(acc[2 * j + 1], pa, b1);
-        mma_f16_16816(acc[2 * j], pl, b0);
-        mma_f16_16816(acc[2 * j + 1], pl, b1);
-      }
-    }
-    __syncthreads();
   }
+  *ok_out = ok;
+  mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+  for (int i = 0; i < S::PPC; ++i)
+    if (src[i] >= 0) bulk_g2s(raw + i * S::PAGE, a.cache + src[i], S::PAGE, bar);
+}
 
-  // ---- epilogue: o = acc / l * v_scale -> fp32 / E4M3 / bf16
-  float lA = l_run[0], lB = l_run[1];
-  lA += __shfl_xor_sync(0xffffffffu, lA, 1);
-  lA += __shfl_xor_sync(0xffffffffu, lA, 2);
-  lB += __shfl_xor_sync(0xffffffffu, lB, 1);
-  lB += __shfl_xor_sync(0xffffffffu, lB, 2);
-  const int rows[2] = {rA, rB};
-  const float ls[2] = {lA, lB};
-#pragma unroll
-  for (int ri = 0; ri < 2; ++ri) {
-    const int r = rows[ri];
-    const int qt = qtok0 + r / G;
-    if (r >= tpt * G || qt >= q_len) continue;
-    const long long obase = ((long long)(q_begin + qt) * a.num_q_heads + h * G + r % G) * D;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-#pragma unroll
-      for (int e2 = 0; e2 < 2; ++e2) {
-        const int d = j * 8 + 2 * t4 + e2;
-        const float o = (ls[ri] > 0.f) ? __fdiv_rn(acc[j][2 * ri + e2], ls[ri]) * v_scale : 0.f;
-        const long long idx = obase + d;
-        if (a.o_f32) a.o_f32[idx] = o;
-        const uint32_t code = f32_to_e4m3(__fdiv_rn(o, o_scale));
-        a.o_fp8[idx] = (uint8_t)code;
-        if (a.o_bf16)
-          reinterpret_cast<__nv_bfloat16*>(a.o_bf16)[idx] =
-              __float2bfloat16_rn(__fmul_rn(e4m3_to_f32(code), o_scale));
-      }
+// Dequantize one chunk (64 keys) from its raw stage into an f16 tile laid out
+// for the MMA: 64-column blocks of [64 keys][64 d] f16, 128-byte rows, the
+// 16-byte chunk j of row n stored at chunk j ^ (n % 8). Keys at or past
+// kv_end, and keys of pages not copied, become zeros. 128 threads.
+template <int D, int BS, int FMT>
+__device__ __forceinline__ void dequant_chunk(const uint8_t* raw, uint32_t ok, uint8_t* tile,
+                                              int key0, int kv_end, int gtid) {
+  using S = PrefillShape<D, BS, FMT>;
+  constexpr int RG = S::kChunk / 8;  // groups of 8 keys
+  const int lane = gtid & 31, gw = gtid >> 5;
+  const int n_lo = lane & 7, c_lo = lane >> 3;  // 8 rows x 4 chunks per warp step
+#pragma unroll 4
+  for (int v = gw; v < 2 * RG * S::DB; v += 4) {
+    const int n = (v % RG) * 8 + n_lo;             // key within the chunk
+    const int c = ((v / RG) & 1) * 4 + c_lo;       // 8-element chunk within the 64-block
+    const int dblk = v / (2 * RG);
+    const int cc = dblk * 8 + c;                   // 8-element chunk of the row
+    const bool valid = (key0 + n < kv_end) && ((ok >> (n / BS)) & 1u);
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (valid && FMT) {  // FP8 row: 8 E4M3 bytes -> 8 f16 (exact)
+      const uint8_t* row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
+      const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * cc);
+      out.x = e4m3x2_to_f16x2(w.x & 0xFFFFu);
+      out.y = e4m3x2_to_f16x2(w.x >> 16);
+      out.z = e4m3x2_to_f16x2(w.y & 0xFFFFu);
+      out.w = e4m3x2_to_f16x2(w.y >> 16);
+    } else if (valid) {
+      const uint8_t* row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
+      const uint32_t codes = ld_shared_u32(smem_u32(row + 4 * cc));
+      const uint32_t sb = row[D / 2 + cc / 2];
+      const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+      out.x = hmul2_u32(e2m1x2_to_f16x2(codes & 0xFFu), s2);
+      out.y = hmul2_u32(e2m1x2_to_f16x2((codes >> 8) & 0xFFu), s2);
+      out.z = hmul2_u32(e2m1x2_to_f16x2((codes >> 16) & 0xFFu), s2);
+      out.w = hmul2_u32(e2m1x2_to_f16x2(codes >> 24), s2);
+    }
+    *reinterpret_cast<uint4*>(tile + dblk * (S::kChunk * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
+        out;
+  }
+}
+
+// The copy + dequant pipeline of one of K (kv = 0) and V (kv = 1).
+template <int D, int BS, int FMT>
+__device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, int h, int nchunk,
+                                        int kv_end, uint8_t* base, uint64_t* bars, Misc* misc,
+                                        uint32_t* status) {
+  using S = PrefillShape<D, BS, FMT>;
+  const int gtid = threadIdx.x - (kv ? kVGroup0 : kKGroup0);
+  const uint32_t bar_id = kv ? kBarV : kBarK;
+  uint8_t* raw = base + (kv ? S::kOffVraw : S::kOffKraw);
+  uint8_t* tiles = base + (kv ? S::kOffV : S::kOffK);
+  uint64_t* raw_full = bars + (kv ? kBarVraw : kBarKraw);
+  uint64_t* full = bars + (kv ? kBarVFull : kBarKFull);
+  uint64_t* empty = bars + (kv ? kBarVEmpty : kBarKEmpty);
+  uint32_t* raw_ok = misc->raw_ok[kv];
+  volatile int* stop = misc->group_stop[kv];
+  int issued = 0;
+  if (gtid == 0) {
+    for (; issued < min(kRawStages, nchunk); ++issued)
+      issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + issued * S::RAW, &raw_full[issued],
+                         &raw_ok[issued], status);
+  }
+  int c = 0;
+  for (; c < nchunk; ++c) {
+    const int st = c % kRawStages;
+    bool ok = wait_bar(&raw_full[st], (uint32_t)((c / kRawStages) & 1), misc, status);
+    if (ok && c >= 2) ok = wait_bar(&empty[c & 1], (uint32_t)(((c >> 1) - 1) & 1), misc, status);
+    if (!ok) stop[c & 1] = 1;  // (the block is aborting: this chunk's data no longer matter)
+    dequant_chunk<D, BS, FMT>(raw + st * S::RAW, raw_ok[st], tiles + (c & 1) * S::TILE,
+                              c * S::kChunk, kv_end, gtid);
+    fence_proxy_async_smem();  // generic writes -> read by the tensor core
+    tc::mbar_arrive(&full[c & 1]);
+    tc::named_sync(bar_id, 128);  // every thread is done with raw stage st
+    if (stop[c & 1]) break;  // (the drain below also covers chunk c's copies)
+    if (gtid == 0 && issued < nchunk) {
+      issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + st * S::RAW, &raw_full[st],
+                         &raw_ok[st], status);
+      ++issued;
+    }
+  }
+  // copies issued but never consumed (stopped early) must land before exit
+  if (gtid == 0) {
+    for (int k = c; k < issued; ++k) {
+      const int st = k % kRawStages;
+      for (int i = 0; i < kMaxPolls; ++i)
+        if (mbar_try_wait(&raw_full[st], (uint32_t)((k / kRawStages) & 1))) break;
     }
   }
 }
 
-template <int D, int BS>
+}  // namespace
+
+template <int D, int BS, int FMT>
+__global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const AttentionArgs a) {
+  using S = PrefillShape<D, BS, FMT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::kOffBar);
+  Misc* misc = reinterpret_cast<Misc*>(base + S::kOffMisc);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int Hkv = a.num_kv_heads, G = a.num_q_heads / Hkv;
+  const int TQ = kRows / G;  // query tokens per CTA
+  const int q_begin = a.qo_indptr[b];
+  const int q_len = a.qo_indptr[b + 1] - q_begin;
+  if (q_len <= 1) return;  // decode rows are served by the decode kernel
+  uint32_t* status = reinterpret_cast<uint32_t*>(a.workspace);
+  if (q_len > (int)gridDim.x * TQ && blockIdx.x == 0 && tid == 0)
+    atomicOr(status, kDevBadQlen);  // rows beyond the grid are not written
+  const int tile_idx = (int)gridDim.x - 1 - (int)blockIdx.x;  // longest (last) tiles first
+  const int qtok0 = tile_idx * TQ;
+  if (qtok0 >= q_len) return;
+  const int L = a.seq_lens[b];
+  const int last_tok = min(q_len - 1, qtok0 + TQ - 1);
+  const int kv_end = max(0, min(min(L, L - q_len + last_tok + 1), a.max_blocks_per_seq * BS));
+  const int nchunk = (kv_end + S::kChunk - 1) / S::kChunk;
+
+  if (tid == 0) {
+    for (int i = 0; i < S::kNumBars; ++i) {
+      const bool many = (i >= kBarKFull && i < kBarKFull + 4) ||
+                        (i >= kBarPFull && i < kBarPFull + kSBufs) || i == kBarQReady;
+      mbar_init(&bars[i], many ? 128u : 1u);
+    }
+    misc->abort = 0;
+    for (int i = 0; i < 3; ++i) misc->group_stop[i][0] = misc->group_stop[i][1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(&misc->tmem_base, S::kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = misc->tmem_base;
+
+  if (warp < 4) {
+    // ------------------------------------------------ Q, softmax, epilogue
+    const int r = tid;
+    const int tok = r / G, g = r % G;
+    const bool row_ok = (r < TQ * G) && (qtok0 + tok < q_len);
+    const int pos = L - q_len + qtok0 + tok;  // absolute position (may be < 0: sees nothing)
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                (long long)(q_begin + qtok0 + tok) * a.q_token_stride +
+                                (long long)(h * G + g) * D;
+    float mx = 0.0f;
+    if (row_ok) {
+#pragma unroll 4
+      for (int i = 0; i < D / 8; ++i) {
+        const uint4 v4 = __ldg(reinterpret_cast<const uint4*>(qrow) + i);
+        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(wv[j] << 16)),
+                               fabsf(__uint_as_float(wv[j] & 0xFFFF0000u))));
+      }
+    }
+    const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
+    const int sh = min(126, max(-126, 15 - ex));
+    const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
+    const float qmult = a.sm_scale * __ldg(a.kv_scales) * kLog2e *
+                        __uint_as_float((uint32_t)(127 - sh) << 23);
+#pragma unroll 1
+    for (int blk = 0; blk < D / 64; ++blk) {
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+        if (row_ok) v4 = __ldg(reinterpret_cast<const uint4*>(qrow + blk * 64) + j);
+        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[4 * j + i] = pack_f16x2(__uint_as_float(wv[i] << 16) * qs,
+                                    __uint_as_float(wv[i] & 0xFFFF0000u) * qs);
+      }
+      tc::tmem_st32(tb + lane_off + S::kColQ + blk * 32, w);
+    }
+    tc::tmem_wait_st();
+    tc::fence_before_sync();
+    tc::mbar_arrive(&bars[kBarQReady]);
+
+    float m_run = -INFINITY, l_run = 0.0f;
+    volatile int* stop = misc->group_stop[2];
+    int done_chunks = 0;
+    constexpr int CH = S::kChunk;
+    for (int c = 0; c < nchunk; ++c) {
+      const int sb = c % kSBufs;
+      const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / kSBufs) & 1), misc, status);
+      if (!ok) stop[c & 1] = 1;
+      tc::named_sync(kBarSoftmax, 128);
+      if (stop[c & 1]) break;
+      tc::fence_after_sync();
+      const uint32_t scol = S::kColS + CH * sb;
+      // logits of this chunk (s0: keys 0..31, s1: keys 32..63 when the chunk has 64)
+      uint32_t s0[32], s1[32];
+      tc::tmem_ld32(tb + lane_off + scol, s0);
+      if constexpr (CH == 64) tc::tmem_ld32(tb + lane_off + scol + 32, s1);
+      tc::tmem_wait_ld();
+      const int key0 = c * CH;
+      const int lim = min(pos + 1, kv_end) - key0;  // keys [key0, key0 + lim) are visible
+      // logits in log2 units, masked in place
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x0 = (i < lim) ? __uint_as_float(s0[i]) * qmult : -INFINITY;
+        s0[i] = __float_as_uint(x0);
+        cmax = fmaxf(cmax, x0);
+        if constexpr (CH == 64) {
+          const float x1 = (32 + i < lim) ? __uint_as_float(s1[i]) * qmult : -INFINITY;
+          s1[i] = __float_as_uint(x1);
+          cmax = fmaxf(cmax, x1);
+        }
+      }
+      // lazy max: move it (and rescale O) only when this chunk exceeds it by > 2^8
+      const bool up = (m_run == -INFINITY) ? (cmax > -INFINITY) : (cmax > m_run + kRescaleThresh);
+      const bool need_o = up && m_run != -INFINITY;  // O holds earlier contributions
+      float alpha = 1.0f;
+      if (up) {
+        const float m_new = fmaxf(m_run, cmax);
+        if (m_run != -INFINITY) alpha = ex2(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      if (__any_sync(0xffffffffu, need_o)) {
+        // every PV MMA so far must be done before O is read and rewritten
+        bool wok = wait_bar(&bars[kBarODone], (uint32_t)((c - 1) & 1), misc, status);
+        if (__all_sync(0xffffffffu, wok)) {
+          tc::fence_after_sync();
+#pragma unroll 1
+          for (int blk = 0; blk < D / 16; ++blk) {
+            uint32_t o[16];
+            tc::tmem_ld16(tb + lane_off + S::kColO + blk * 16, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tc::tmem_st16(tb + lane_off + S::kColO + blk * 16, o);
+          }
+          tc::tmem_wait_st();
+        } else {
+          stop[(c + 1) & 1] = 1;  // read after the next chunk's barrier
+        }
+      }
+      // P = exp2(x - m) as f16 hi (columns scol .. scol + CH/2 - 1, keys in pairs)
+      // and lo = f16(P - hi) (the next CH/2 columns), 16 columns at a time
+      const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // all x are -inf then: P = 0
+      float psum = 0.0f;
+#pragma unroll
+      for (int part = 0; part < CH / 32; ++part) {
+        const uint32_t(&xs)[32] = part ? s1 : s0;
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(__uint_as_float(xs[2 * i]) - mu);
+          const float p1 = ex2(__uint_as_float(xs[2 * i + 1]) - mu);
+          psum += p0 + p1;
+          hw[i] = pack_f16x2(p0, p1);
+          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+          lw[i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
+        }
+        tc::tmem_st16(tb + lane_off + scol + 16 * part, hw);
+        tc::tmem_st16(tb + lane_off + scol + CH / 2 + 16 * part, lw);
+      }
+      l_run += psum;
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[kBarPFull + sb]);
+      done_chunks = c + 1;
+    }
+
+    // ---- epilogue: o = O / l * v_scale -> fp32 / E4M3 / bf16
+    // O is final once every MMA has completed: the one-time barrier the MMA
+    // thread commits after its last PV (a per-chunk barrier could still have
+    // two chunks outstanding here, which a parity wait cannot tell apart)
+    bool have_o = false;
+    if (done_chunks == nchunk && nchunk > 0) {
+      const bool ok = wait_bar(&bars[kBarFin], 0u, misc, status);
+      have_o = __all_sync(0xffffffffu, ok);
+    }
+    tc::fence_after_sync();
+    const float v_scale = __ldg(a.kv_scales + 1);
+    const float o_scale = __ldg(a.o_scale);
+    const float inv_os = 1.0f / o_scale;
+    const float scl = (l_run > 0.0f) ? v_scale / l_run : 0.0f;
+    const long long obase =
+        ((long long)(q_begin + qtok0 + tok) * a.num_q_heads + h * G + g) * D;
+    const bool vec8 = (reinterpret_cast<uintptr_t>(a.o_fp8) & 15) == 0;
+    const bool vec16 = (reinterpret_cast<uintptr_t>(a.o_bf16) & 15) == 0;
+    const bool vec32 = (reinterpret_cast<uintptr_t>(a.o_f32) & 15) == 0;
+#pragma unroll 1
+    for (int blk = 0; blk < D / 32; ++blk) {
+      uint32_t o[32];
+      if (have_o) {  // (warp-uniform: every lane loads its row)
+        tc::tmem_ld32(tb + lane_off + S::kColO + blk * 32, o);
+        tc::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (row_ok) {
+      float f[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(o[i]) * scl;
+      const long long idx = obase + blk * 32;
+      if (a.o_f32) {
+        if (vec32) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(a.o_f32 + idx)[i] =
+                make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            reinterpret_cast<float2*>(a.o_f32 + idx)[i] = make_float2(f[2 * i], f[2 * i + 1]);
+        }
+      }
+      uint32_t codes[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) codes[i] = f32x2_to_e4m3x2(f[2 * i] * inv_os, f[2 * i + 1] * inv_os);
+      if (vec8) {
+        uint4* dst = reinterpret_cast<uint4*>(a.o_fp8 + idx);
+        dst[0] = make_uint4(codes[0] | codes[1] << 16, codes[2] | codes[3] << 16,
+                            codes[4] | codes[5] << 16, codes[6] | codes[7] << 16);
+        dst[1] = make_uint4(codes[8] | codes[9] << 16, codes[10] | codes[11] << 16,
+                            codes[12] | codes[13] << 16, codes[14] | codes[15] << 16);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          reinterpret_cast<uint16_t*>(a.o_fp8 + idx)[i] = (uint16_t)codes[i];
+      }
+      if (a.o_bf16) {
+        uint32_t bw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t h2 = e4m3x2_to_f16x2(codes[i]);
+          const float2 ff = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(ff.x, o_scale), __fmul_rn(ff.y, o_scale));
+          bw[i] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(a.o_bf16) + idx;
+        if (vec16) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<uint4*>(ob)[i] = make_uint4(bw[4 * i], bw[4 * i + 1], bw[4 * i + 2], bw[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) reinterpret_cast<uint32_t*>(ob)[i] = bw[i];
+        }
+      }
+      }  // row_ok
+      __syncwarp();
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issue (one thread)
+    if (lane == 0 && nchunk > 0) {
+      constexpr int CH = S::kChunk;
+      constexpr uint32_t kIdescS = tc::idesc_f16(kRows, CH, false);
+      constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
+      const uint32_t kbase = smem_u32(base + S::kOffK), vbase = smem_u32(base + S::kOffV);
+      bool ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
+      // order: S_0, S_1, PV_0, S_2, PV_1, ... ; S_c overwrites the TMEM buffer
+      // of P_{c-3} only after the PV MMAs that read it have completed
+      for (int c = 0; ok && c <= nchunk; ++c) {
+        if (c < nchunk) {
+          const int sb = c % kSBufs;
+          ok = wait_bar(&bars[kBarKFull + (c & 1)], (uint32_t)((c >> 1) & 1), misc, status);
+          if (ok && c >= kSBufs)
+            ok = wait_bar(&bars[kBarPFree + sb], (uint32_t)((c / kSBufs - 1) & 1), misc, status);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t kt = kbase + (c & 1) * S::TILE;
+          const uint32_t dS = tb + S::kColS + CH * sb;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t desc =
+                tc::sw128_desc(kt + (kk >> 2) * (CH * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+          }
+          tc::commit(&bars[kBarKEmpty + (c & 1)]);
+          tc::commit(&bars[kBarSFull + sb]);
+        }
+        if (c >= 1) {
+          const int j = c - 1, pb = j % kSBufs;
+          ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((j / kSBufs) & 1), misc, status);
+          if (ok) ok = wait_bar(&bars[kBarVFull + (j & 1)], (uint32_t)((j >> 1) & 1), misc, status);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t vt = vbase + (j & 1) * S::TILE;
+          const uint32_t pS = tb + S::kColS + CH * pb;
+#pragma unroll
+          for (int i = 0; i < CH / 16; ++i) {
+            const uint64_t desc = tc::sw128_desc(vt + i * 2048, CH * 128, 1024);
+            tc::mma_ts(tb + S::kColO, pS + i * 8, desc, kIdescPV, j > 0 || i > 0);
+            tc::mma_ts(tb + S::kColO, pS + CH / 2 + i * 8, desc, kIdescPV, true);
+          }
+          tc::commit(&bars[kBarVEmpty + (j & 1)]);
+          tc::commit(&bars[kBarPFree + pb]);
+          tc::commit(&bars[kBarODone]);
+        }
+      }
+      // every MMA issued has completed before TMEM is released
+      tc::commit(&bars[kBarFin]);
+      for (int i = 0; i < kMaxPolls; ++i)
+        if (mbar_try_wait(&bars[kBarFin], 0u)) break;
+    }
+    __syncwarp();
+  } else if (tid < kVGroup0) {
+    kv_role<D, BS, FMT>(a, 0, b, h, nchunk, kv_end, base, bars, misc, status);
+  } else {
+    kv_role<D, BS, FMT>(a, 1, b, h, nchunk, kv_end, base, bars, misc, status);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tb, S::kTmemCols);
+  }
+}
+
+template <int D, int BS, int FMT>
 static cudaError_t launch_prefill_t(const AttentionArgs& a, cudaStream_t stream) {
-  using S = PrefillShape<D, BS>;
+  using S = PrefillShape<D, BS, FMT>;
   const size_t smem = S::smem_bytes();
-  auto kern = prefill_attention_kernel<D, BS>;
+  auto kern = prefill_attention_kernel<D, BS, FMT>;
   // the attribute is set once per (device, context), under a lock
   static std::mutex attr_mutex;
   static unsigned long long attr_ctx[64] = {0};
@@ -319,15 +607,17 @@ static cudaError_t launch_prefill_t(const AttentionArgs& a, cudaStream_t stream)
     }
   }
   const int G = a.num_q_heads / a.num_kv_heads;
-  const int tpt = kRows / G;
-  dim3 grid((a.max_q_len + tpt - 1) / tpt, a.num_kv_heads, a.num_seqs);
-  kern<<<grid, kPWarps * 32, smem, stream>>>(a);
+  const int TQ = kRows / G;
+  dim3 grid((a.max_q_len + TQ - 1) / TQ, a.num_kv_heads, a.num_seqs);
+  kern<<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_attention(const AttentionArgs& a, cudaStream_t stream) {
-#define NVFP4_PREFILL_CASE(DD, BB) \
-  if (a.head_size == DD && a.block_size == BB) return launch_prefill_t<DD, BB>(a, stream);
+#define NVFP4_PREFILL_CASE(DD, BB)                                             \
+  if (a.head_size == DD && a.block_size == BB)                                 \
+    return a.kv_format ? launch_prefill_t<DD, BB, 1>(a, stream)                \
+                       : launch_prefill_t<DD, BB, 0>(a, stream);
   NVFP4_PREFILL_CASE(64, 16)
   NVFP4_PREFILL_CASE(64, 32)
   NVFP4_PREFILL_CASE(128, 16)

@@ -91,6 +91,88 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
+// ------------------------------------------------------------ NVFP4 encode
+// E2M1 codes of fl32(x_i / S) for 8 values (element 2j in the low nibble of
+// byte j). Fast path: y = x * rcp.approx(S) is within 2^-21 (relative) of
+// x / S (the reciprocal is within 1 ulp, the product rounds by half an ulp),
+// and so is fl32(x / S). If y * (1 - 2^-20) and y * (1 + 2^-20) give the same
+// code, no rounding threshold of the E2M1 grid lies between them, and the
+// conversion is monotone, so fl32(x / S) has that code as well. Otherwise
+// (x / S within ~1e-6 of a threshold, exact ties included) the quotient is
+// formed with IEEE division. S must be a positive normal number; above
+// 2^100 the reciprocal nears the subnormal range, where its 1-ulp bound no
+// longer holds, so such scales always divide.
+__device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S) {
+  if (S > 1.2676506e30f) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
+    return f32x8_to_e2m1x8(q);
+  }
+  float r;
+  asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(S));
+  float lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float y = x[i] * r;
+    lo[i] = y * 0.99999904632568359375f;  // 1 - 2^-20
+    hi[i] = y * 1.00000095367431640625f;  // 1 + 2^-20
+  }
+  const uint32_t c_lo = f32x8_to_e2m1x8(lo);
+  const uint32_t c_hi = f32x8_to_e2m1x8(hi);
+  if (c_lo == c_hi) return c_lo;
+  float q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
+  return f32x8_to_e2m1x8(q);
+}
+
+// E4M3 byte of fl32(a / b) (RNE, satfinite). Fast path as for the codes: the
+// quotient from the approximate reciprocal is within 2^-21 of fl32(a / b);
+// when both ends of the +-2^-20 bracket encode to the same byte, so does
+// fl32(a / b). Otherwise, and for b outside [2^-100, 2^100] or a non-finite
+// a, the quotient is formed with IEEE division.
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float b) {
+  if (b >= 7.8886091e-31f && b <= 1.2676506e30f && a <= 3.4028235e38f) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(b));
+    const float y = a * r;
+    const uint32_t two = f32x2_to_e4m3x2(y * 0.99999904632568359375f, y * 1.00000095367431640625f);
+    if ((two & 0xFFu) == (two >> 8)) return two & 0xFFu;
+  }
+  return f32_to_e4m3(__fdiv_rn(a, b));
+}
+
+
+// One group of 16 values (element 2j in the low nibble of byte j): the E4M3
+// block scale sb = E4M3(fl32(amax / fl32(6 g))) (returned) and the E2M1 codes
+// of fl32(x_i / fl32(E4M3(sb) g)) in c0 (elements 0..7) and c1 (8..15); every
+// code is 0 when that effective scale is 0. Bit-exact with IEEE fp32 division.
+__device__ __forceinline__ uint32_t quantize_group16(const float (&x)[16], float g, uint32_t& c0,
+                                                     uint32_t& c1) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const uint32_t sb = e4m3_of_quotient(amax, __fmul_rn(6.0f, g));
+  const float S = __fmul_rn(e4m3_to_f32(sb), g);
+  c0 = 0u;
+  c1 = 0u;
+  if (S >= 1.17549435e-38f) {
+    c0 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x), S);
+    c1 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x + 8), S);
+  } else if (S > 0.0f) {  // subnormal effective scale: divide exactly
+    float q0[8], q1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q0[i] = __fdiv_rn(x[i], S);
+      q1[i] = __fdiv_rn(x[8 + i], S);
+    }
+    c0 = f32x8_to_e2m1x8(q0);
+    c1 = f32x8_to_e2m1x8(q1);
+  }
+  return sb;
+}
+
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));

@@ -21,6 +21,6 @@ AttentionArgs attention_args(const void* q, int64_t q_token_stride, int64_t num_
 int check_attention(const AttentionArgs& a, bool* nothing_to_do);
 int launch_attention(const AttentionArgs& a, cudaStream_t stream);
 int cuda_status(cudaError_t e);
-int decode_warps(int head_size, int block_size, int num_seqs, int group);
+int decode_warps(int head_size, int block_size, int num_seqs, int group, int kv_format);
 
 }  // namespace nvfp4kv

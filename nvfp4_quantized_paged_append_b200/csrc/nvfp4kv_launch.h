@@ -21,6 +21,16 @@ struct QuantizeAppendArgs {
   const float* k_scale;
   const float* v_scale;
   uint32_t* device_status;
+  int kv_format;  // 0: NVFP4 rows, 1: FP8-E4M3 rows
+};
+
+struct ActivationArgs {
+  const void* x;  // bf16 [rows][row_stride]
+  int64_t rows, cols, row_stride;
+  const float* global_scale_inv;
+  uint8_t* out_fp4;  // [rows][cols / 2]
+  uint8_t* out_sf;   // swizzled or [rows][cols / 16]
+  bool swizzled;
 };
 
 struct DequantArgs {
@@ -57,6 +67,13 @@ struct AttentionArgs {
   float* o_f32;   // may be null
   void* workspace;
   uint32_t flags;  // NVFP4_ATTN_* launch flags (0: none)
+  // fused append (decode only; k_new == nullptr: none): bf16 [num_seqs][Hkv][D]
+  // rows of every sequence's newest token, quantized and written to position
+  // seq_lens[b] - 1 of the cache by the decode kernel itself
+  const void* k_new;
+  const void* v_new;
+  int64_t k_new_stride, v_new_stride;  // token strides in elements
+  int kv_format;  // 0: NVFP4 rows (D/2 + D/16 bytes), 1: FP8-E4M3 rows (D bytes)
 };
 
 // Decode split-KV: at most kDecodeWarps warps in the whole grid; every warp
@@ -96,6 +113,7 @@ cudaError_t current_context_id(unsigned long long* id);
 
 cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t stream);
 cudaError_t launch_dequantize_paged(const DequantArgs& a, cudaStream_t stream);
+cudaError_t launch_quantize_activation(const ActivationArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_attention(const AttentionArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_attention(const AttentionArgs& a, cudaStream_t stream);
 // A one-block kernel that arms an mbarrier for 16 bytes no copy will deliver,

@@ -11,61 +11,12 @@
 //
 // Mapping: one CTA per token, one thread per 16-element block of a row (two
 // 16-byte bf16 loads, one E4M3 scale byte, 8 bytes of packed codes).
+#include <algorithm>
+
 #include "nvfp4kv_device.cuh"
 #include "nvfp4kv_launch.h"
 
 namespace nvfp4kv {
-
-// E2M1 codes of fl32(x_i / S) for 8 values (element 2j in the low nibble of
-// byte j). Fast path: y = x * rcp.approx(S) is within 2^-21 (relative) of
-// x / S (the reciprocal is within 1 ulp, the product rounds by half an ulp),
-// and so is fl32(x / S). If y * (1 - 2^-20) and y * (1 + 2^-20) give the same
-// code, no rounding threshold of the E2M1 grid lies between them, and the
-// conversion is monotone, so fl32(x / S) has that code as well. Otherwise
-// (x / S within ~1e-6 of a threshold, exact ties included) the quotient is
-// formed with IEEE division. S must be a positive normal number; above
-// 2^100 the reciprocal nears the subnormal range, where its 1-ulp bound no
-// longer holds, so such scales always divide.
-__device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S) {
-  if (S > 1.2676506e30f) {
-    float q[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
-    return f32x8_to_e2m1x8(q);
-  }
-  float r;
-  asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(S));
-  float lo[8], hi[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float y = x[i] * r;
-    lo[i] = y * 0.99999904632568359375f;  // 1 - 2^-20
-    hi[i] = y * 1.00000095367431640625f;  // 1 + 2^-20
-  }
-  const uint32_t c_lo = f32x8_to_e2m1x8(lo);
-  const uint32_t c_hi = f32x8_to_e2m1x8(hi);
-  if (c_lo == c_hi) return c_lo;
-  float q[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], S);
-  return f32x8_to_e2m1x8(q);
-}
-
-// E4M3 byte of fl32(a / b) (RNE, satfinite). Fast path as for the codes: the
-// quotient from the approximate reciprocal is within 2^-21 of fl32(a / b);
-// when both ends of the +-2^-20 bracket encode to the same byte, so does
-// fl32(a / b). Otherwise, and for b outside [2^-100, 2^100] or a non-finite
-// a, the quotient is formed with IEEE division.
-__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float b) {
-  if (b >= 7.8886091e-31f && b <= 1.2676506e30f && a <= 3.4028235e38f) {
-    float r;
-    asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(b));
-    const float y = a * r;
-    const uint32_t two = f32x2_to_e4m3x2(y * 0.99999904632568359375f, y * 1.00000095367431640625f);
-    if ((two & 0xFFu) == (two >> 8)) return two & 0xFFu;
-  }
-  return f32_to_e4m3(__fdiv_rn(a, b));
-}
 
 // One CTA per new token: its K and V rows of every kv head, one thread per
 // 16-element block (two 16-byte bf16 loads, one scale, 8 bytes of codes). A
@@ -108,26 +59,9 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
       x[2 * i] = __uint_as_float(wv[i] << 16);
       x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
     const float g = kv == 0 ? gk : gv;
-    const uint32_t sb = e4m3_of_quotient(amax, __fmul_rn(6.0f, g));
-    const float S = __fmul_rn(e4m3_to_f32(sb), g);
-    uint32_t c0 = 0u, c1 = 0u;  // S == 0: every code 0
-    if (S >= 1.17549435e-38f) {
-      c0 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x), S);
-      c1 = e2m1_codes_div(*reinterpret_cast<const float(*)[8]>(x + 8), S);
-    } else if (S > 0.0f) {  // subnormal effective scale: divide exactly
-      float q0[8], q1[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        q0[i] = __fdiv_rn(x[i], S);
-        q1[i] = __fdiv_rn(x[8 + i], S);
-      }
-      c0 = f32x8_to_e2m1x8(q0);
-      c1 = f32x8_to_e2m1x8(q1);
-    }
+    uint32_t c0, c1;
+    const uint32_t sb = quantize_group16(x, g, c0, c1);
     uint8_t* dst =
         cache + (((blk * 2 + kv) * num_kv_heads + h) * (int64_t)block_size + off) * F;
     if constexpr (F % 8 == 0) {  // rows 8-byte aligned
@@ -137,6 +71,138 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
       reinterpret_cast<uint32_t*>(dst + 8 * j)[1] = c1;
     }
     dst[D / 2 + j] = (uint8_t)sb;
+  }
+}
+
+// Grid-stride writer: thread `idx` of a block owns group idx % TPR of row
+// idx / TPR (K rows first, then V rows) of every token the block visits
+// (blockDim.x == 2 * num_kv_heads * D / 16). The next token's slot and input
+// words are loaded before the current token is quantized, so the two memory
+// latencies of a token (its slot, then its rows) overlap with other work.
+// FP8 = false: NVFP4 rows; true: FP8-E4M3 rows.
+template <int D, bool FP8>
+__global__ void __launch_bounds__(1024) quantize_append_stream_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    int64_t k_stride, int64_t v_stride, int num_kv_heads, uint8_t* __restrict__ cache,
+    int64_t num_tokens, int64_t num_blocks, int bs_log2, const int64_t* __restrict__ slot_mapping,
+    const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+    uint32_t* __restrict__ status) {
+  constexpr int TPR = D / 16;
+  constexpr int F = FP8 ? D : D / 2 + D / 16;
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  const int idx = threadIdx.x;
+  const int rr = idx / TPR, j = idx % TPR;
+  const int kv = rr >= num_kv_heads ? 1 : 0;
+  const int h = rr - kv * num_kv_heads;
+  const __nv_bfloat16* src0 = (kv == 0 ? k : v) + h * D + j * 16;
+  const int64_t stride = kv == 0 ? k_stride : v_stride;
+  const float g = __ldg(kv == 0 ? k_scale : v_scale);
+  const int block_size = 1 << bs_log2;
+  int64_t t = blockIdx.x;
+  int64_t slot = -1;
+  uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
+  if (t < num_tokens) {
+    slot = __ldg(slot_mapping + t);
+    r0 = __ldg(reinterpret_cast<const uint4*>(src0 + t * stride));
+    r1 = __ldg(reinterpret_cast<const uint4*>(src0 + t * stride) + 1);
+  }
+  while (t < num_tokens) {
+    const int64_t tn = t + gridDim.x;
+    int64_t slot_n = -1;
+    uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+    if (tn < num_tokens) {  // rows exist for every token: loaded before the slot is known
+      slot_n = __ldg(slot_mapping + tn);
+      n0 = __ldg(reinterpret_cast<const uint4*>(src0 + tn * stride));
+      n1 = __ldg(reinterpret_cast<const uint4*>(src0 + tn * stride) + 1);
+    }
+    if (slot >= (num_blocks << bs_log2)) {
+      if (idx == 0 && status) atomicOr(status, kDevBadSlot);
+    } else if (slot >= 0) {
+      const int64_t blk = slot >> bs_log2;
+      const int off = (int)(slot & (block_size - 1));
+      uint8_t* dst =
+          cache + (((blk * 2 + kv) * num_kv_heads + h) * (int64_t)block_size + off) * F;
+      const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      if constexpr (FP8) {
+        uint32_t out[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t b0 = e4m3_of_quotient(__uint_as_float(wv[2 * i] << 16), g);
+          const uint32_t b1 = e4m3_of_quotient(__uint_as_float(wv[2 * i] & 0xFFFF0000u), g);
+          const uint32_t b2 = e4m3_of_quotient(__uint_as_float(wv[2 * i + 1] << 16), g);
+          const uint32_t b3 = e4m3_of_quotient(__uint_as_float(wv[2 * i + 1] & 0xFFFF0000u), g);
+          out[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        }
+        *reinterpret_cast<uint4*>(dst + 16 * j) = make_uint4(out[0], out[1], out[2], out[3]);
+      } else {
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[2 * i] = __uint_as_float(wv[i] << 16);
+          x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        uint32_t c0, c1;
+        const uint32_t sb = quantize_group16(x, g, c0, c1);
+        if constexpr (F % 8 == 0) {
+          *reinterpret_cast<uint2*>(dst + 8 * j) = make_uint2(c0, c1);
+        } else {
+          reinterpret_cast<uint32_t*>(dst + 8 * j)[0] = c0;
+          reinterpret_cast<uint32_t*>(dst + 8 * j)[1] = c1;
+        }
+        dst[D / 2 + j] = (uint8_t)sb;
+      }
+    }
+    t = tn;
+    slot = slot_n;
+    r0 = n0;
+    r1 = n1;
+  }
+}
+
+// FP8-E4M3 rows (the comparison format): code = E4M3 RNE satfinite of
+// fl32(x / g) per element (same bracketed reciprocal fast path, IEEE division
+// near rounding thresholds), D bytes per row in the same HND page layout.
+template <int D>
+__global__ void __launch_bounds__(256) quantize_append_fp8_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    int64_t k_stride, int64_t v_stride, int num_kv_heads, uint8_t* __restrict__ cache,
+    int64_t num_blocks, int bs_log2, const int64_t* __restrict__ slot_mapping,
+    const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+    uint32_t* __restrict__ status) {
+  constexpr int TPR = D / 16;
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  const int64_t t = blockIdx.x;
+  const int64_t slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= (num_blocks << bs_log2)) {
+    if (threadIdx.x == 0 && status) atomicOr(status, kDevBadSlot);
+    return;
+  }
+  const int64_t blk = slot >> bs_log2;
+  const int off = (int)(slot & ((1 << bs_log2) - 1));
+  const int block_size = 1 << bs_log2;
+  const float gk = __ldg(k_scale), gv = __ldg(v_scale);
+  const int nthr = 2 * num_kv_heads * TPR;
+  for (int idx = threadIdx.x; idx < nthr; idx += blockDim.x) {
+    const int rr = idx / TPR, j = idx % TPR;
+    const int kv = rr >= num_kv_heads ? 1 : 0;
+    const int h = rr - kv * num_kv_heads;
+    const __nv_bfloat16* src = (kv == 0 ? k + t * k_stride : v + t * v_stride) + h * D + j * 16;
+    const uint4 r0 = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    const float g = kv == 0 ? gk : gv;
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t b0 = e4m3_of_quotient(__uint_as_float(wv[2 * i] << 16), g);
+      const uint32_t b1 = e4m3_of_quotient(__uint_as_float(wv[2 * i] & 0xFFFF0000u), g);
+      const uint32_t b2 = e4m3_of_quotient(__uint_as_float(wv[2 * i + 1] << 16), g);
+      const uint32_t b3 = e4m3_of_quotient(__uint_as_float(wv[2 * i + 1] & 0xFFFF0000u), g);
+      out[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+    uint8_t* dst = cache + (((blk * 2 + kv) * num_kv_heads + h) * (int64_t)block_size + off) * D;
+    *reinterpret_cast<uint4*>(dst + 16 * j) = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -178,16 +244,55 @@ cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t str
   const int bs_log2 = (a.block_size == 16) ? 4 : 5;  // validated: 16 or 32
   // one thread per 16-element block of the token's 2 * num_kv_heads rows
   const int rows_threads = 2 * a.num_kv_heads * (a.head_size / 16);
+  const auto* k = static_cast<const __nv_bfloat16*>(a.k);
+  const auto* v = static_cast<const __nv_bfloat16*>(a.v);
+  if (rows_threads % 32 == 0 && rows_threads <= 1024) {
+    // grid-stride blocks, as many as are resident at once (tokens per block
+    // rise with the batch)
+    int dev = 0, sms = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+#define NVFP4_STREAM_CASE(DD)                                                                  \
+  case DD: {                                                                                   \
+    auto kern = a.kv_format ? quantize_append_stream_kernel<DD, true>                          \
+                            : quantize_append_stream_kernel<DD, false>;                        \
+    int per_sm = 1;                                                                            \
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, rows_threads, 0);       \
+    if (err != cudaSuccess) return err;                                                        \
+    const long long resident = (long long)sms * std::max(1, per_sm);                           \
+    const unsigned grid = (unsigned)std::min<long long>(a.num_tokens, resident);               \
+    kern<<<grid, rows_threads, 0, stream>>>(k, v, a.k_token_stride, a.v_token_stride,          \
+                                            a.num_kv_heads, a.cache, a.num_tokens,             \
+                                            a.num_blocks, bs_log2, a.slot_mapping, a.k_scale,  \
+                                            a.v_scale, a.device_status);                       \
+    break;                                                                                     \
+  }
+    switch (a.head_size) {
+      NVFP4_STREAM_CASE(64)
+      NVFP4_STREAM_CASE(128)
+      NVFP4_STREAM_CASE(256)
+      default:
+        return cudaErrorInvalidValue;
+    }
+#undef NVFP4_STREAM_CASE
+    return cudaGetLastError();
+  }
+  // many heads: one block per token, threads loop over the token's groups
   const int block = rows_threads <= 128 ? 128 : 256;
   if (a.num_tokens > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)a.num_tokens;
-  const auto* k = static_cast<const __nv_bfloat16*>(a.k);
-  const auto* v = static_cast<const __nv_bfloat16*>(a.v);
 #define NVFP4_WRITER_CASE(DD)                                                                  \
   case DD:                                                                                     \
-    quantize_append_kernel<DD><<<grid, block, 0, stream>>>(                                    \
-        k, v, a.k_token_stride, a.v_token_stride, a.num_kv_heads, a.cache, a.num_blocks,       \
-        bs_log2, a.slot_mapping, a.k_scale, a.v_scale, a.device_status);                       \
+    if (a.kv_format)                                                                           \
+      quantize_append_fp8_kernel<DD><<<grid, block, 0, stream>>>(                              \
+          k, v, a.k_token_stride, a.v_token_stride, a.num_kv_heads, a.cache, a.num_blocks,     \
+          bs_log2, a.slot_mapping, a.k_scale, a.v_scale, a.device_status);                     \
+    else                                                                                       \
+      quantize_append_kernel<DD><<<grid, block, 0, stream>>>(                                  \
+          k, v, a.k_token_stride, a.v_token_stride, a.num_kv_heads, a.cache, a.num_blocks,     \
+          bs_log2, a.slot_mapping, a.k_scale, a.v_scale, a.device_status);                     \
     break;
   switch (a.head_size) {
     NVFP4_WRITER_CASE(64)

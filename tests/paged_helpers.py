@@ -25,21 +25,24 @@ def dev_scalar(x: float, device="cuda") -> torch.Tensor:
     return torch.tensor([x], dtype=torch.float32, device=device)
 
 
-def build_gpu_cache(w: wl.PagedWorkload, scales, device="cuda", sentinel: int | None = None):
-    """Device HND cache written by the library's writer, token by sequence."""
+def build_gpu_cache(w: wl.PagedWorkload, scales, device="cuda", sentinel: int | None = None,
+                    fp8: bool = False):
+    """Device HND cache written by the library's writer, token by sequence
+    (fp8: an FP8-E4M3 cache)."""
     k_scale, v_scale, _ = scales
-    cache = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, device)
+    alloc = nk.alloc_fp8_kv_cache if fp8 else nk.alloc_kv_cache
+    cache = alloc(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, device)
     if sentinel is not None:
         cache.fill_(sentinel)
     ks, vs = dev_scalar(k_scale, device), dev_scalar(v_scale, device)
     for b in range(w.num_seqs):
         k, v = wl.seq_kv(w, b, device)
         slots = torch.from_numpy(w.slots_for_seq(b)).to(device)
-        nk.quantize_append_paged(k, v, cache, slots, ks, vs)
+        nk.quantize_append_paged(k, v, cache, slots, ks, vs, fp8=fp8)
     return cache
 
 
-def oracle_case(w: wl.PagedWorkload, seqs, scales, device="cuda", rows=None):
+def oracle_case(w: wl.PagedWorkload, seqs, scales, device="cuda", rows=None, fp8=False):
     """Oracle inputs for the listed sequences: compact cache + block table.
 
     rows: optional {b: [query row indices]} for prefill sequences; each listed
@@ -56,15 +59,16 @@ def oracle_case(w: wl.PagedWorkload, seqs, scales, device="cuda", rows=None):
         blocks += [int(x) for x in w.block_table[b, : -(-int(w.seq_lens[b]) // w.block_size)]]
     remap = {blk: i for i, blk in enumerate(dict.fromkeys(blocks))}
     nb = len(remap)
-    cache = np.zeros((nb, 2, w.num_kv_heads, w.block_size, w.full_dim), np.uint8)
+    row_bytes = w.head_size if fp8 else w.full_dim
+    cache = np.zeros((nb, 2, w.num_kv_heads, w.block_size, row_bytes), np.uint8)
+    writer = oracle.fp8kv_quantize_append_paged if fp8 else oracle.quantize_append_paged
     for b in seqs:
         k, v = wl.seq_kv(w, b, device)
         L = int(w.seq_lens[b])
         n = np.arange(L)
         loc = np.array([remap[int(x)] for x in w.block_table[b, n // w.block_size]], np.int64)
         slots = loc * w.block_size + n % w.block_size
-        oracle.quantize_append_paged(u16(k), u16(v), cache, slots.astype(np.int64), k_scale,
-                                     v_scale, w.block_size)
+        writer(u16(k), u16(v), cache, slots.astype(np.int64), k_scale, v_scale, w.block_size)
     tables, lens, qrows, out_index = [], [], [], []
     for b in seqs:
         L = int(w.seq_lens[b])
@@ -84,16 +88,17 @@ def oracle_case(w: wl.PagedWorkload, seqs, scales, device="cuda", rows=None):
     for i, t in enumerate(tables):
         bt[i, : len(t)] = t
     return dict(cache=cache, block_table=bt, seq_lens=np.array(lens, np.int32),
-                q=np.ascontiguousarray(np.stack(qrows)), out_index=out_index)
+                q=np.ascontiguousarray(np.stack(qrows)), out_index=out_index, fp8=fp8)
 
 
 def run_oracle(case, scales):
     k_scale, v_scale, o_scale = scales
     return oracle.paged_attention(case["q"], case["cache"], case["block_table"], case["seq_lens"],
-                                  None, k_scale, v_scale, 0.0, o_scale)
+                                  None, k_scale, v_scale, 0.0, o_scale,
+                                  kv_format=oracle.KV_FP8 if case.get("fp8") else oracle.KV_NVFP4)
 
 
-def run_gpu_attention(w: wl.PagedWorkload, cache, scales, device="cuda", q=None):
+def run_gpu_attention(w: wl.PagedWorkload, cache, scales, device="cuda", q=None, fp8=False):
     k_scale, v_scale, o_scale = scales
     q = wl.queries(w, device) if q is None else q
     tq = q.shape[0]
@@ -106,7 +111,7 @@ def run_gpu_attention(w: wl.PagedWorkload, cache, scales, device="cuda", q=None)
     qo = None if w.is_decode else torch.from_numpy(w.qo_indptr).to(device)
     kvs = torch.tensor([k_scale, v_scale], dtype=torch.float32, device=device)
     nk.paged_attention(q, cache, bt, sl, kvs, o8, dev_scalar(o_scale, device), ws, qo_indptr=qo,
-                       max_q_len=w.max_q_len, o_bf16=o16, o_f32=o32)
+                       max_q_len=w.max_q_len, o_bf16=o16, o_f32=o32, fp8=fp8)
     torch.cuda.synchronize()
     return o8, o16, o32, ws
 

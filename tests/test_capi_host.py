@@ -191,3 +191,45 @@ def test_binding_rejects_bad_attention_tensors(L):
             run(o_fp8=torch.zeros((2, 4, 64), dtype=torch.uint8))  # output shape
         with pytest.raises(ValueError):
             run(cache=torch.zeros((4, 2, 2, 16, 70), dtype=torch.uint8))  # not a full_dim
+
+
+def test_fused_decode_append_validation(L):
+    """The fused decode step rejects bad arguments before any CUDA call."""
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+
+    def call(**kw):
+        a = dict(q=fake, qs=16 * 128, hq=16, k=fake, v=fake, ks=8 * 128, vs=8 * 128, cache=fake,
+                 nb=100, bs=16, hkv=8, d=128, bt=fake, mb=10, sl=fake, B=4, kvs=fake,
+                 o8=fake, os=fake, ws=fake, wsb=1 << 30, flags=0)
+        a.update(kw)
+        return L.nvfp4_paged_decode_append(a["q"], a["qs"], a["hq"], a["k"], a["v"], a["ks"],
+                                           a["vs"], a["cache"], a["nb"], a["bs"], a["hkv"],
+                                           a["d"], a["bt"], a["mb"], a["sl"], a["B"], a["kvs"],
+                                           0.0, a["o8"], a["os"], None, None, a["ws"], a["wsb"],
+                                           a["flags"], None)
+    assert call(k=None) == nk.NVFP4_ERR_INVALID_ARG
+    assert call(v=None) == nk.NVFP4_ERR_INVALID_ARG
+    assert call(ks=8 * 128 - 8) == nk.NVFP4_ERR_INVALID_ARG        # stride below a token row
+    assert call(k=P(0x1008)) == nk.NVFP4_ERR_INVALID_ARG            # rows not 16-byte aligned
+    assert call(flags=0x2) == nk.NVFP4_ERR_INVALID_ARG
+    assert call(wsb=16) == nk.NVFP4_ERR_WORKSPACE
+    assert call(d=96) == nk.NVFP4_ERR_UNSUPPORTED
+    assert call(B=0) == nk.NVFP4_OK                                 # empty batch: nothing to do
+
+
+def test_activation_validation(L):
+    """The activation quantizer rejects bad shapes and pointers before any CUDA
+    call; its scale-buffer size follows the padded tile layout."""
+    fake = ctypes.c_void_p(0x1000)
+    q = L.nvfp4_quantize_activation
+    assert q(None, 4, 96, 96, fake, fake, fake, 1, None) == nk.NVFP4_ERR_INVALID_ARG
+    assert q(fake, 4, 100, 104, fake, fake, fake, 1, None) == nk.NVFP4_ERR_INVALID_ARG   # cols % 16
+    assert q(fake, 4, 96, 90, fake, fake, fake, 1, None) == nk.NVFP4_ERR_INVALID_ARG     # stride < cols
+    assert q(fake, 4, 96, 100, fake, fake, fake, 1, None) == nk.NVFP4_ERR_INVALID_ARG    # stride % 8
+    assert q(ctypes.c_void_p(0x1008), 4, 96, 96, fake, fake, fake, 1, None) == \
+        nk.NVFP4_ERR_INVALID_ARG                                                         # x alignment
+    assert q(fake, 0, 96, 96, None, None, None, 1, None) == nk.NVFP4_OK                   # no rows
+    assert nk.activation_sf_bytes(200, 96, True) == 256 * 8
+    assert nk.activation_sf_bytes(200, 96, False) == 200 * 6
+    assert nk.activation_sf_bytes(4, 100, True) == 0

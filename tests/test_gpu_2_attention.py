@@ -76,6 +76,12 @@ EDGE = [
     (128, 16, 8, 2, [5], [9]),                              # q_len > L: early rows see nothing
     (128, 16, 12, 4, [100, 700, 2500], None),               # G = 3: odd group, lo columns cross lanes
     (64, 16, 12, 2, [90, 1300], None),                      # G = 6: separate lo fragments
+    # chunked prefill on the tensor cores: M = 128 rows of (token, head)
+    (128, 32, 4, 4, [700, 129], [300, 129]),                # G = 1: 128 tokens per tile
+    (128, 16, 12, 4, [515, 64], [200, 3]),                  # G = 3: 42 tokens (126 rows)
+    (256, 16, 40, 8, [333, 20], [90, 7]),                   # G = 5: 25 tokens (125 rows)
+    (256, 16, 64, 8, [3000, 1], [700, 1]),                  # G = 8, many 64-key chunks
+    (64, 32, 8, 4, [64, 65, 191], [64, 65, 2]),             # chunk and page edges, D 64
 ]
 
 
@@ -132,6 +138,28 @@ def test_bad_block_id_flagged_no_fault():
     assert st == nk.NVFP4_ERR_DEVICE_BOUNDS and bits & nk.DEV_BAD_BLOCK
     assert nk.read_device_status(out[3]) == (nk.NVFP4_OK, 0)
     assert torch.isfinite(out[2]).all()
+
+
+def test_prefill_bad_block_id_flagged_no_fault():
+    """An out-of-range block id inside a prefill range: its page is skipped (no
+    fault), the status reads back NVFP4_ERR_DEVICE_BOUNDS, outputs are finite,
+    and rows whose causal window ends before that page match the oracle."""
+    w = wl.custom_workload("pf_badblk", 8, 16, 8, 128, 16, [400], [300])
+    scales = wl.global_scales(w, DEV)
+    cache = build_gpu_cache(w, scales, DEV)
+    good = int(w.block_table[0, 20])
+    w.block_table[0, 20] = w.num_blocks + 77     # keys 320..335
+    out = run_gpu_attention(w, cache, scales, DEV)
+    st, bits = nk.read_device_status(out[3])
+    assert st == nk.NVFP4_ERR_DEVICE_BOUNDS and bits & nk.DEV_BAD_BLOCK
+    assert torch.isfinite(out[2]).all()
+    # rows at positions < 320 never see the bad page
+    rows = {0: [0, 1, 50, 150, 219]}             # positions 100 .. 319
+    w.block_table[0, 20] = good                  # (the oracle's rows never read that page)
+    case = oracle_case(w, [0], scales, DEV, rows=rows)
+    o64, r8, _ = run_oracle(case, scales)
+    idx = case["out_index"]
+    check_rows(out[2].cpu().numpy()[idx].reshape(-1, w.head_size), o64.reshape(-1, w.head_size))
 
 
 def test_query_range_beyond_max_q_len_flagged():
