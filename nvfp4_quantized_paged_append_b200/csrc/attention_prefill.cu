@@ -44,8 +44,12 @@ namespace nvfp4kv {
 
 namespace {
 constexpr int kRows = 128;   // M of every MMA: (query token, head) rows per CTA
-constexpr int kSBufs = 3;    // S/P buffers in TMEM
+constexpr int kSBufs = 4;    // S/P buffers in TMEM
+constexpr int kSlots = 3;    // f16 K (and V) tile slots
 constexpr int kRawStages = 3;
+// block ids of a CTA's pages held in shared memory (longer ranges read them
+// from the block table as they go)
+constexpr int kMaxIds = 4096;
 constexpr int kThreads = 13 * 32;
 constexpr int kMmaWarp = 4;
 constexpr int kKGroup0 = 5 * 32;  // first thread of the K warps
@@ -61,15 +65,14 @@ constexpr size_t kMinSmem = 120 * 1024;
 enum : int {
   kBarKraw = 0,                   // [3] K raw stage filled (expect_tx)
   kBarVraw = kRawStages,          // [3] V raw stage filled
-  kBarKFull = 2 * kRawStages,     // [2] K tile dequantized (128 arrivals)
-  kBarVFull = kBarKFull + 2,      // [2] V tile dequantized (128 arrivals)
-  kBarKEmpty = kBarVFull + 2,     // [2] S MMAs that read the K tile done (commit)
-  kBarVEmpty = kBarKEmpty + 2,    // [2] PV MMAs that read the V tile done (commit)
-  kBarSFull = kBarVEmpty + 2,     // [3] S chunk in TMEM (commit)
-  kBarPFull = kBarSFull + kSBufs, // [3] P chunk in TMEM (128 arrivals)
-  kBarPFree = kBarPFull + kSBufs, // [3] PV MMAs that read a P buffer done (commit)
-  kBarODone = kBarPFree + kSBufs, // PV MMAs of a chunk done (commit)
-  kBarQReady = kBarODone + 1,     // Q rows in TMEM (128 arrivals)
+  kBarKFull = 2 * kRawStages,     // [3] K tile dequantized (128 arrivals)
+  kBarVFull = kBarKFull + kSlots, // [3] V tile dequantized (128 arrivals)
+  kBarKEmpty = kBarVFull + kSlots,  // [3] S MMAs that read the K tile done (commit)
+  kBarVEmpty = kBarKEmpty + kSlots, // [3] PV MMAs that read the V tile done (commit)
+  kBarSFull = kBarVEmpty + kSlots,  // [4] S chunk in TMEM (commit)
+  kBarPFull = kBarSFull + kSBufs, // [4] P chunk in TMEM (128 arrivals)
+  kBarPFree = kBarPFull + kSBufs, // [4] PV MMAs that read a P buffer done (commit)
+  kBarQReady = kBarPFree + kSBufs,  // Q rows in TMEM (128 arrivals)
   kBarFin = kBarQReady + 1,       // every MMA issued done (commit)
   kNumBarriers = kBarFin + 1
 };
@@ -77,7 +80,7 @@ enum : int {
 template <int D, int BS, int FMT>
 struct PrefillShape {
   // keys per chunk: N of S = Q K^T and the K-extent of O += P V (32 at head
-  // size 256, where three S/P buffers must fit beside O and Q in TMEM)
+  // size 256, where four S/P buffers must fit beside O and Q in TMEM)
   static constexpr int kChunk = D == 256 ? 32 : 64;
   static constexpr int F = FMT ? D : D / 2 + D / 16;  // row bytes: NVFP4, or FP8 (FMT = 1)
   static constexpr int PAGE = BS * F;          // bytes of one (block, K|V, head) page
@@ -85,18 +88,19 @@ struct PrefillShape {
   static constexpr int RAW = kChunk * F;       // cache bytes of a chunk (K or V)
   static constexpr int TILE = kChunk * D * 2;  // f16 tile of a chunk
   static constexpr int DB = D / 64;            // 64-column blocks of a tile
-  // TMEM columns: O [0, D), S/P buffers [D, D + 3 chunk), Q after them (D/2)
+  // TMEM columns: O [0, D), S/P buffers [D, D + 4 chunk), Q after them (D/2)
   static constexpr uint32_t kColO = 0, kColS = D, kColQ = D + kSBufs * kChunk;
   static constexpr uint32_t kTmemCols = (kColQ + D / 2 <= 256) ? 256u : 512u;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = 2 * TILE;
-  static constexpr int kOffKraw = 4 * TILE;
+  static constexpr int kOffV = kSlots * TILE;
+  static constexpr int kOffKraw = 2 * kSlots * TILE;
   static constexpr int kOffVraw = kOffKraw + kRawStages * RAW;
   static constexpr int kOffBar = kOffVraw + kRawStages * RAW;
   static constexpr int kNumBars = kNumBarriers;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kBytes = kOffMisc + 64;
+  static constexpr int kOffIds = kOffMisc + 64;             // [2][kMaxIds] block ids (K, V)
+  static constexpr int kBytes = kOffIds + 2 * kMaxIds * 4;
   static size_t smem_bytes() {
     const size_t need = (size_t)kBytes + 1024;  // + alignment of the base
     return need > kMinSmem ? need : kMinSmem;
@@ -137,7 +141,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* m
 template <int D, int BS, int FMT>
 __device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h, int kv, int c,
                                             int kv_end, uint8_t* raw, uint64_t* bar,
-                                            uint32_t* ok_out, uint32_t* status) {
+                                            uint32_t* ok_out, uint32_t* status, const int* ids) {
   using S = PrefillShape<D, BS, FMT>;
   const int Hkv = a.num_kv_heads;
   uint32_t ok = 0, bytes = 0;
@@ -147,7 +151,8 @@ __device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h
     const int p = c * S::PPC + i;
     src[i] = -1;
     if (p * BS < kv_end && p < a.max_blocks_per_seq) {
-      const long long blk = __ldg(a.block_table + (long long)b * a.max_blocks_per_seq + p);
+      const long long blk =
+          ids ? ids[p] : __ldg(a.block_table + (long long)b * a.max_blocks_per_seq + p);
       if (blk >= 0 && blk < a.num_blocks) {
         src[i] = ((blk * 2 + kv) * Hkv + h) * (long long)S::PAGE;
         ok |= 1u << i;
@@ -220,27 +225,38 @@ __device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, i
   uint64_t* empty = bars + (kv ? kBarVEmpty : kBarKEmpty);
   uint32_t* raw_ok = misc->raw_ok[kv];
   volatile int* stop = misc->group_stop[kv];
+  // the block ids of this CTA's pages, loaded once (coalesced) into shared memory
+  const int npages = min((kv_end + BS - 1) / BS, a.max_blocks_per_seq);
+  int* ids = nullptr;
+  if (npages <= kMaxIds) {
+    ids = reinterpret_cast<int*>(base + S::kOffIds) + kv * kMaxIds;
+    const int* row = a.block_table + (long long)b * a.max_blocks_per_seq;
+    for (int p = gtid; p < npages; p += 128) ids[p] = __ldg(row + p);
+    tc::named_sync(bar_id, 128);
+  }
   int issued = 0;
   if (gtid == 0) {
     for (; issued < min(kRawStages, nchunk); ++issued)
       issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + issued * S::RAW, &raw_full[issued],
-                         &raw_ok[issued], status);
+                              &raw_ok[issued], status, ids);
   }
   int c = 0;
   for (; c < nchunk; ++c) {
     const int st = c % kRawStages;
     bool ok = wait_bar(&raw_full[st], (uint32_t)((c / kRawStages) & 1), misc, status);
-    if (ok && c >= 2) ok = wait_bar(&empty[c & 1], (uint32_t)(((c >> 1) - 1) & 1), misc, status);
+    const int slot = c % kSlots;
+    if (ok && c >= kSlots)
+      ok = wait_bar(&empty[slot], (uint32_t)((c / kSlots - 1) & 1), misc, status);
     if (!ok) stop[c & 1] = 1;  // (the block is aborting: this chunk's data no longer matter)
-    dequant_chunk<D, BS, FMT>(raw + st * S::RAW, raw_ok[st], tiles + (c & 1) * S::TILE,
+    dequant_chunk<D, BS, FMT>(raw + st * S::RAW, raw_ok[st], tiles + slot * S::TILE,
                               c * S::kChunk, kv_end, gtid);
     fence_proxy_async_smem();  // generic writes -> read by the tensor core
-    tc::mbar_arrive(&full[c & 1]);
+    tc::mbar_arrive(&full[slot]);
     tc::named_sync(bar_id, 128);  // every thread is done with raw stage st
     if (stop[c & 1]) break;  // (the drain below also covers chunk c's copies)
     if (gtid == 0 && issued < nchunk) {
       issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + st * S::RAW, &raw_full[st],
-                         &raw_ok[st], status);
+                              &raw_ok[st], status, ids);
       ++issued;
     }
   }
@@ -285,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
 
   if (tid == 0) {
     for (int i = 0; i < S::kNumBars; ++i) {
-      const bool many = (i >= kBarKFull && i < kBarKFull + 4) ||
+      const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kSlots) ||
                         (i >= kBarPFull && i < kBarPFull + kSBufs) || i == kBarQReady;
       mbar_init(&bars[i], many ? 128u : 1u);
     }
@@ -365,18 +381,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       const int key0 = c * CH;
       const int lim = min(pos + 1, kv_end) - key0;  // keys [key0, key0 + lim) are visible
       // logits in log2 units, masked in place
-      float cmax = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // (independent chains)
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float x0 = (i < lim) ? __uint_as_float(s0[i]) * qmult : -INFINITY;
         s0[i] = __float_as_uint(x0);
-        cmax = fmaxf(cmax, x0);
+        mx4[i & 3] = fmaxf(mx4[i & 3], x0);
         if constexpr (CH == 64) {
           const float x1 = (32 + i < lim) ? __uint_as_float(s1[i]) * qmult : -INFINITY;
           s1[i] = __float_as_uint(x1);
-          cmax = fmaxf(cmax, x1);
+          mx4[i & 3] = fmaxf(mx4[i & 3], x1);
         }
       }
+      const float cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       // lazy max: move it (and rescale O) only when this chunk exceeds it by > 2^8
       const bool up = (m_run == -INFINITY) ? (cmax > -INFINITY) : (cmax > m_run + kRescaleThresh);
       const bool need_o = up && m_run != -INFINITY;  // O holds earlier contributions
@@ -389,7 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       }
       if (__any_sync(0xffffffffu, need_o)) {
         // every PV MMA so far must be done before O is read and rewritten
-        bool wok = wait_bar(&bars[kBarODone], (uint32_t)((c - 1) & 1), misc, status);
+        // (P-free of chunk c - 1: PV_{c-1} and, in issue order, every PV before it
+        // done; that barrier is at most one phase behind here)
+        bool wok = wait_bar(&bars[kBarPFree + (c - 1) % kSBufs], (uint32_t)(((c - 1) / kSBufs) & 1),
+                            misc, status);
         if (__all_sync(0xffffffffu, wok)) {
           tc::fence_after_sync();
 #pragma unroll 1
@@ -409,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       // P = exp2(x - m) as f16 hi (columns scol .. scol + CH/2 - 1, keys in pairs)
       // and lo = f16(P - hi) (the next CH/2 columns), 16 columns at a time
       const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // all x are -inf then: P = 0
-      float psum = 0.0f;
+      float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int part = 0; part < CH / 32; ++part) {
         const uint32_t(&xs)[32] = part ? s1 : s0;
@@ -418,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2(__uint_as_float(xs[2 * i]) - mu);
           const float p1 = ex2(__uint_as_float(xs[2 * i + 1]) - mu);
-          psum += p0 + p1;
+          ps4[i & 3] += p0 + p1;
           hw[i] = pack_f16x2(p0, p1);
           const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
           lw[i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
@@ -426,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         tc::tmem_st16(tb + lane_off + scol + 16 * part, hw);
         tc::tmem_st16(tb + lane_off + scol + CH / 2 + 16 * part, lw);
       }
-      l_run += psum;
+      l_run += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
       tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[kBarPFull + sb]);
@@ -523,45 +543,47 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
       const uint32_t kbase = smem_u32(base + S::kOffK), vbase = smem_u32(base + S::kOffV);
       bool ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
-      // order: S_0, S_1, PV_0, S_2, PV_1, ... ; S_c overwrites the TMEM buffer
-      // of P_{c-3} only after the PV MMAs that read it have completed
-      for (int c = 0; ok && c <= nchunk; ++c) {
-        if (c < nchunk) {
-          const int sb = c % kSBufs;
-          ok = wait_bar(&bars[kBarKFull + (c & 1)], (uint32_t)((c >> 1) & 1), misc, status);
-          if (ok && c >= kSBufs)
-            ok = wait_bar(&bars[kBarPFree + sb], (uint32_t)((c / kSBufs - 1) & 1), misc, status);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t kt = kbase + (c & 1) * S::TILE;
-          const uint32_t dS = tb + S::kColS + CH * sb;
+      // S = Q K^T of chunk j into TMEM buffer j % 4 (after the PV MMAs that read
+      // the P held there, chunk j - 4, have completed)
+      auto issue_s = [&](int j) -> bool {
+        const int sb = j % kSBufs, slot = j % kSlots;
+        bool k = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / kSlots) & 1), misc, status);
+        if (k && j >= kSBufs)
+          k = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / kSBufs - 1) & 1), misc, status);
+        if (!k) return false;
+        tc::fence_after_sync();
+        const uint32_t kt = kbase + slot * S::TILE;
+        const uint32_t dS = tb + S::kColS + CH * sb;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t desc =
-                tc::sw128_desc(kt + (kk >> 2) * (CH * 128) + (kk & 3) * 32, 16, 1024);
-            tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
-          }
-          tc::commit(&bars[kBarKEmpty + (c & 1)]);
-          tc::commit(&bars[kBarSFull + sb]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t desc =
+              tc::sw128_desc(kt + (kk >> 2) * (CH * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
         }
-        if (c >= 1) {
-          const int j = c - 1, pb = j % kSBufs;
-          ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((j / kSBufs) & 1), misc, status);
-          if (ok) ok = wait_bar(&bars[kBarVFull + (j & 1)], (uint32_t)((j >> 1) & 1), misc, status);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t vt = vbase + (j & 1) * S::TILE;
-          const uint32_t pS = tb + S::kColS + CH * pb;
+        tc::commit(&bars[kBarKEmpty + slot]);
+        tc::commit(&bars[kBarSFull + sb]);
+        return true;
+      };
+      // order: S_0, S_1, then S_{c+2}, PV_c for c = 0, 1, ...: two S chunks are
+      // queued on the tensor core while the softmax of chunk c runs
+      for (int j = 0; ok && j < min(2, nchunk); ++j) ok = issue_s(j);
+      for (int c = 0; ok && c < nchunk; ++c) {
+        if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
+        const int pb = c % kSBufs, slot = c % kSlots;
+        ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / kSBufs) & 1), misc, status);
+        if (ok) ok = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / kSlots) & 1), misc, status);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t vt = vbase + slot * S::TILE;
+        const uint32_t pS = tb + S::kColS + CH * pb;
 #pragma unroll
-          for (int i = 0; i < CH / 16; ++i) {
-            const uint64_t desc = tc::sw128_desc(vt + i * 2048, CH * 128, 1024);
-            tc::mma_ts(tb + S::kColO, pS + i * 8, desc, kIdescPV, j > 0 || i > 0);
-            tc::mma_ts(tb + S::kColO, pS + CH / 2 + i * 8, desc, kIdescPV, true);
-          }
-          tc::commit(&bars[kBarVEmpty + (j & 1)]);
-          tc::commit(&bars[kBarPFree + pb]);
-          tc::commit(&bars[kBarODone]);
+        for (int i = 0; i < CH / 16; ++i) {
+          const uint64_t desc = tc::sw128_desc(vt + i * 2048, CH * 128, 1024);
+          tc::mma_ts(tb + S::kColO, pS + i * 8, desc, kIdescPV, c > 0 || i > 0);
+          tc::mma_ts(tb + S::kColO, pS + CH / 2 + i * 8, desc, kIdescPV, true);
         }
+        tc::commit(&bars[kBarVEmpty + slot]);
+        tc::commit(&bars[kBarPFree + pb]);
       }
       // every MMA issued has completed before TMEM is released
       tc::commit(&bars[kBarFin]);
