@@ -219,22 +219,6 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
   return v;
 }
 
-// The four E2M1 pairs held in the bytes of w -> four f16x2 (low nibble ->
-// low half). Unpacking with mov.b32 lets each conversion read its byte
-// directly, without shifts.
-__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&r)[4]) {
-  asm("{\n"
-      ".reg .b8 b0, b1, b2, b3;\n"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n"
-      "}\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-      : "r"(w));
-}
-
 // Per-lane byte offsets inside a 16-token tile (constant for the kernel).
 struct LaneOffsets {
   uint32_t k0, k1;              // K data segment of rows g8, g8+8

@@ -87,7 +87,6 @@ struct PrefillShape {
   static constexpr int PPC = kChunk >= BS ? kChunk / BS : 1;  // pages per chunk
   static constexpr int RAW = kChunk * F;       // cache bytes of a chunk (K or V)
   static constexpr int TILE = kChunk * D * 2;  // f16 tile of a chunk
-  static constexpr int DB = D / 64;            // 64-column blocks of a tile
   // TMEM columns: O [0, D), S/P buffers [D, D + 4 chunk), Q after them (D/2)
   static constexpr uint32_t kColO = 0, kColS = D, kColQ = D + kSBufs * kChunk;
   static constexpr uint32_t kTmemCols = (kColQ + D / 2 <= 256) ? 256u : 512u;
@@ -169,44 +168,64 @@ __device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h
     if (src[i] >= 0) bulk_g2s(raw + i * S::PAGE, a.cache + src[i], S::PAGE, bar);
 }
 
-// Dequantize one chunk (64 keys) from its raw stage into an f16 tile laid out
-// for the MMA: 64-column blocks of [64 keys][64 d] f16, 128-byte rows, the
-// 16-byte chunk j of row n stored at chunk j ^ (n % 8). Keys at or past
-// kv_end, and keys of pages not copied, become zeros. 128 threads.
+// Dequantize one chunk from its raw stage into an f16 tile laid out for the
+// MMA: 64-column blocks of [chunk keys][64 d] f16, 128-byte rows, the 16-byte
+// chunk j of row n stored at chunk j ^ (n % 8). A thread converts one scale
+// group (16 elements of one key: 8 code bytes and their E4M3 scale) per step;
+// a warp step covers 8 keys x 4 groups, so both the code loads and the tile
+// stores are free of bank conflicts. Keys at or past kv_end, and keys of pages
+// not copied, become zeros. 128 threads.
 template <int D, int BS, int FMT>
-__device__ __forceinline__ void dequant_chunk(const uint8_t* raw, uint32_t ok, uint8_t* tile,
-                                              int key0, int kv_end, int gtid) {
+__device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_t tile, int key0,
+                                              int kv_end, int gtid) {
   using S = PrefillShape<D, BS, FMT>;
-  constexpr int RG = S::kChunk / 8;  // groups of 8 keys
+  constexpr int KB = S::kChunk / 8;  // blocks of 8 keys
+  constexpr int GB = D / 64;         // blocks of 4 groups (one 64-column tile block each)
   const int lane = gtid & 31, gw = gtid >> 5;
-  const int n_lo = lane & 7, c_lo = lane >> 3;  // 8 rows x 4 chunks per warp step
-#pragma unroll 4
-  for (int v = gw; v < 2 * RG * S::DB; v += 4) {
-    const int n = (v % RG) * 8 + n_lo;             // key within the chunk
-    const int c = ((v / RG) & 1) * 4 + c_lo;       // 8-element chunk within the 64-block
-    const int dblk = v / (2 * RG);
-    const int cc = dblk * 8 + c;                   // 8-element chunk of the row
+  const int n_lo = lane & 7, g_lo = lane >> 3;
+#pragma unroll
+  for (int blk = gw; blk < KB * GB; blk += 4) {
+    const int n = (blk % KB) * 8 + n_lo;  // key within the chunk
+    const int dblk = blk / KB;            // 64-column block
+    const int g = dblk * 4 + g_lo;        // scale group of the row
     const bool valid = (key0 + n < kv_end) && ((ok >> (n / BS)) & 1u);
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (valid && FMT) {  // FP8 row: 8 E4M3 bytes -> 8 f16 (exact)
-      const uint8_t* row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
-      const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * cc);
-      out.x = e4m3x2_to_f16x2(w.x & 0xFFFFu);
-      out.y = e4m3x2_to_f16x2(w.x >> 16);
-      out.z = e4m3x2_to_f16x2(w.y & 0xFFFFu);
-      out.w = e4m3x2_to_f16x2(w.y >> 16);
-    } else if (valid) {
-      const uint8_t* row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
-      const uint32_t codes = ld_shared_u32(smem_u32(row + 4 * cc));
-      const uint32_t sb = row[D / 2 + cc / 2];
-      const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
-      out.x = hmul2_u32(e2m1x2_to_f16x2(codes & 0xFFu), s2);
-      out.y = hmul2_u32(e2m1x2_to_f16x2((codes >> 8) & 0xFFu), s2);
-      out.z = hmul2_u32(e2m1x2_to_f16x2((codes >> 16) & 0xFFu), s2);
-      out.w = hmul2_u32(e2m1x2_to_f16x2(codes >> 24), s2);
+    const uint32_t row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
+    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+    if (valid) {
+      if constexpr (FMT) {  // FP8 row: 16 E4M3 bytes -> 16 f16 (exact)
+        uint32_t w[4];
+        lds_v4(row + 16 * g, w);
+        lo.x = e4m3x2_to_f16x2(w[0] & 0xFFFFu);
+        lo.y = e4m3x2_to_f16x2(w[0] >> 16);
+        lo.z = e4m3x2_to_f16x2(w[1] & 0xFFFFu);
+        lo.w = e4m3x2_to_f16x2(w[1] >> 16);
+        hi.x = e4m3x2_to_f16x2(w[2] & 0xFFFFu);
+        hi.y = e4m3x2_to_f16x2(w[2] >> 16);
+        hi.z = e4m3x2_to_f16x2(w[3] & 0xFFFFu);
+        hi.w = e4m3x2_to_f16x2(w[3] >> 16);
+      } else {  // NVFP4 row: 8 code bytes x one E4M3 scale -> 16 f16 (exact)
+        uint32_t c0, c1;
+        if constexpr (S::F % 8 == 0) {
+          lds_v2(row + 8 * g, c0, c1);
+        } else {
+          c0 = ld_shared_u32(row + 8 * g);
+          c1 = ld_shared_u32(row + 8 * g + 4);
+        }
+        const uint32_t sb = lds_b8(row + D / 2 + g);
+        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+        uint32_t x[4], y[4];
+        e2m1x8_to_f16x2x4(c0, x);
+        e2m1x8_to_f16x2x4(c1, y);
+        lo = make_uint4(hmul2_u32(x[0], s2), hmul2_u32(x[1], s2), hmul2_u32(x[2], s2),
+                        hmul2_u32(x[3], s2));
+        hi = make_uint4(hmul2_u32(y[0], s2), hmul2_u32(y[1], s2), hmul2_u32(y[2], s2),
+                        hmul2_u32(y[3], s2));
+      }
     }
-    *reinterpret_cast<uint4*>(tile + dblk * (S::kChunk * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
-        out;
+    const uint32_t dst = tile + dblk * (S::kChunk * 128) + n * 128;
+    const int c = 2 * g_lo;  // 16-byte chunks c, c + 1 of the 128-byte row
+    sts_v4(dst + ((c ^ (n & 7)) << 4), lo);
+    sts_v4(dst + (((c + 1) ^ (n & 7)) << 4), hi);
   }
 }
 
@@ -248,8 +267,8 @@ __device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, i
     if (ok && c >= kSlots)
       ok = wait_bar(&empty[slot], (uint32_t)((c / kSlots - 1) & 1), misc, status);
     if (!ok) stop[c & 1] = 1;  // (the block is aborting: this chunk's data no longer matter)
-    dequant_chunk<D, BS, FMT>(raw + st * S::RAW, raw_ok[st], tiles + slot * S::TILE,
-                              c * S::kChunk, kv_end, gtid);
+    dequant_chunk<D, BS, FMT>(smem_u32(raw + st * S::RAW), raw_ok[st],
+                              smem_u32(tiles + slot * S::TILE), c * S::kChunk, kv_end, gtid);
     fence_proxy_async_smem();  // generic writes -> read by the tensor core
     tc::mbar_arrive(&full[slot]);
     tc::named_sync(bar_id, 128);  // every thread is done with raw stage st

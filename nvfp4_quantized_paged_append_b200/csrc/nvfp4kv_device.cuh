@@ -32,10 +32,12 @@ __device__ __forceinline__ void grid_dependency_wait() {
 constexpr int kMaxWaitIters = 1 << 24;
 
 // ------------------------------------------------------------ conversions
+// (pure register-to-register asm, not volatile: the compiler may schedule
+// and combine it like ordinary arithmetic)
 // Pack 8 fp32 values into 8 E2M1 nibbles: x[2j] -> low nibble of byte j.
 __device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float x[8]) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n"
       ".reg .b8 q0, q1, q2, q3;\n"
       "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n"
@@ -53,14 +55,14 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float x[8]) {
 // fp32 -> E4M3 byte (RNE, satfinite), returned in the low 8 bits.
 __device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
   uint16_t r;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(0.0f), "f"(x));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(0.0f), "f"(x));
   return r & 0xFFu;
 }
 
 // two fp32 -> two E4M3 bytes: lo in bits 0..7, hi in bits 8..15.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t r;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
 
@@ -68,14 +70,30 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   uint32_t out;
   uint16_t in = (uint16_t)two_bytes;
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(out) : "h"(in));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(out) : "h"(in));
   return out;
+}
+
+// The four E2M1 pairs held in the bytes of w -> four f16x2 (low nibble ->
+// low half). Unpacking with mov.b32 lets each conversion read its byte
+// directly, without shifts.
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&r)[4]) {
+  asm("{\n"
+      ".reg .b8 b0, b1, b2, b3;\n"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n"
+      "}\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(w));
 }
 
 // E2M1 pair in one byte (low nibble -> lo half) -> f16x2; exact.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n"
       ".reg .b8 b;\n"
       "cvt.u8.u32 b, %1;\n"
@@ -294,6 +312,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+__device__ __forceinline__ void lds_v2(uint32_t addr, uint32_t& x, uint32_t& y) {
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(x), "=r"(y) : "r"(addr));
+}
+__device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t (&w)[4]) {
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t lds_b8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_v4(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
