@@ -61,7 +61,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--profile", choices=["attention", "append", "step", "activation"],
+    p.add_argument("--profile", choices=["attention", "append", "step", "activation", "prefill"],
                    default=None,
                    help="kernel-only mode for profilers: set up, then launch the chosen "
                         "kernel --steps times (no timing, no JSON)")
@@ -994,7 +994,14 @@ def run_profile(args):
         for _ in range(args.steps):
             nk.quantize_append_paged(k, v, cache, slots, ks, vs)
     else:
-        w = wl.make_workload(args.workload)
+        if args.profile == "prefill":
+            # a small chunked-prefill batch with the mixed batch's shapes: 2
+            # sequences of 512 causal queries over 2560 keys, 64 q / 8 kv heads,
+            # head size 256, block size 16 (512 CTAs)
+            w = wl.custom_workload("prefill_small", 11, 64, 8, 256, 16, [2560, 2560],
+                                   [512, 512], outliers="x20")
+        else:
+            w = wl.make_workload(args.workload)
         scales = wl.global_scales(w, dev)
         cache = nk.alloc_kv_cache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_size, dev)
         ks = torch.tensor([scales[0]], device=dev)

@@ -44,9 +44,9 @@ namespace nvfp4kv {
 
 namespace {
 constexpr int kRows = 128;   // M of every MMA: (query token, head) rows per CTA
-constexpr int kSBufs = 4;    // S/P buffers in TMEM
-constexpr int kSlots = 3;    // f16 K (and V) tile slots
-constexpr int kRawStages = 3;
+constexpr int kMaxSBufs = 4;  // S/P buffers in TMEM (at most)
+constexpr int kMaxSlots = 3;  // f16 K (and V) tile slots (at most)
+constexpr int kMaxRawStages = 3;  // raw page stages per K and V (at most)
 // block ids of a CTA's pages held in shared memory (longer ranges read them
 // from the block table as they go)
 constexpr int kMaxIds = 4096;
@@ -64,24 +64,30 @@ constexpr size_t kMinSmem = 120 * 1024;
 // Barrier slots.
 enum : int {
   kBarKraw = 0,                   // [3] K raw stage filled (expect_tx)
-  kBarVraw = kRawStages,          // [3] V raw stage filled
-  kBarKFull = 2 * kRawStages,     // [3] K tile dequantized (128 arrivals)
-  kBarVFull = kBarKFull + kSlots, // [3] V tile dequantized (128 arrivals)
-  kBarKEmpty = kBarVFull + kSlots,  // [3] S MMAs that read the K tile done (commit)
-  kBarVEmpty = kBarKEmpty + kSlots, // [3] PV MMAs that read the V tile done (commit)
-  kBarSFull = kBarVEmpty + kSlots,  // [4] S chunk in TMEM (commit)
-  kBarPFull = kBarSFull + kSBufs, // [4] P chunk in TMEM (128 arrivals)
-  kBarPFree = kBarPFull + kSBufs, // [4] PV MMAs that read a P buffer done (commit)
-  kBarQReady = kBarPFree + kSBufs,  // Q rows in TMEM (128 arrivals)
+  kBarVraw = kMaxRawStages,       // [3] V raw stage filled
+  kBarKFull = 2 * kMaxRawStages,     // [3] K tile dequantized (128 arrivals)
+  kBarVFull = kBarKFull + kMaxSlots, // [3] V tile dequantized (128 arrivals)
+  kBarKEmpty = kBarVFull + kMaxSlots,  // [3] S MMAs that read the K tile done (commit)
+  kBarVEmpty = kBarKEmpty + kMaxSlots, // [3] PV MMAs that read the V tile done (commit)
+  kBarSFull = kBarVEmpty + kMaxSlots,  // [4] S chunk in TMEM (commit)
+  kBarPFull = kBarSFull + kMaxSBufs, // [4] P chunk in TMEM (128 arrivals)
+  kBarPFree = kBarPFull + kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
+  kBarQReady = kBarPFree + kMaxSBufs,  // Q rows in TMEM (128 arrivals)
   kBarFin = kBarQReady + 1,       // every MMA issued done (commit)
   kNumBarriers = kBarFin + 1
 };
 
 template <int D, int BS, int FMT>
 struct PrefillShape {
-  // keys per chunk: N of S = Q K^T and the K-extent of O += P V (32 at head
-  // size 256, where four S/P buffers must fit beside O and Q in TMEM)
-  static constexpr int kChunk = D == 256 ? 32 : 64;
+  // keys per chunk: N of S = Q K^T and the K-extent of O += P V. S/P buffers
+  // in TMEM: four, or two at head size 256 (where O and Q take 384 of the 512
+  // columns); f16 K and V tile slots: three, or two at head size 256 (shared
+  // memory).
+  static constexpr int kChunk = 64;
+  static constexpr int kSBufs = D == 256 ? 2 : 4;
+  static constexpr int kSlots = D == 256 ? 2 : 3;
+  // raw page stages per K and V: three, or two for FP8 rows at head size 256
+  static constexpr int kRawStages = (FMT && D == 256) ? 2 : 3;
   static constexpr int F = FMT ? D : D / 2 + D / 16;  // row bytes: NVFP4, or FP8 (FMT = 1)
   static constexpr int PAGE = BS * F;          // bytes of one (block, K|V, head) page
   static constexpr int PPC = kChunk >= BS ? kChunk / BS : 1;  // pages per chunk
@@ -107,6 +113,9 @@ struct PrefillShape {
   static_assert(RAW % 16 == 0 && PAGE % 16 == 0, "bulk copies move 16-byte multiples");
   static_assert(TILE % 1024 == 0, "swizzle atoms sit on 1024-byte boundaries");
   static_assert(kColQ + D / 2 <= 512, "TMEM budget");
+  static_assert(kSBufs <= kMaxSBufs && kSlots <= kMaxSlots && kRawStages <= kMaxRawStages,
+                "barrier arrays");
+  static_assert(kBytes + 1024 <= 227 * 1024, "shared memory per block");
   static_assert(kChunk % BS == 0, "a chunk holds whole pages");
   static_assert(kOffMisc + 64 <= kBytes, "misc block fits");
 };
@@ -119,15 +128,20 @@ struct Misc {
   // slot is written again only at chunk c + 2, after every thread of the group
   // has passed the barrier of chunk c + 1
   int group_stop[3][2];
-  uint32_t raw_ok[2][kRawStages];  // per raw stage: bit i = page i of the chunk was copied
+  uint32_t raw_ok[2][kMaxRawStages];  // per raw stage: bit i = page i of the chunk was copied
 };
 
 // Bounded wait that also gives up once another role has aborted the block.
+// A waiter off the critical path (relaxed) sleeps briefly between polls, so
+// that it leaves the issue slots of its SM sub-partition to the softmax and
+// MMA warps there.
+constexpr unsigned kRelaxedSleepNs = 64;
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* misc,
-                                         uint32_t* status) {
+                                         uint32_t* status, bool relaxed = false) {
   for (int i = 0; i < kMaxPolls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 127) == 127 && *reinterpret_cast<volatile int*>(&misc->abort)) return false;
+    if (relaxed) __nanosleep(kRelaxedSleepNs);
   }
   atomicOr(status, kDevTimeout);
   *reinterpret_cast<volatile int*>(&misc->abort) = 1;
@@ -183,7 +197,7 @@ __device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_
   constexpr int GB = D / 64;         // blocks of 4 groups (one 64-column tile block each)
   const int lane = gtid & 31, gw = gtid >> 5;
   const int n_lo = lane & 7, g_lo = lane >> 3;
-#pragma unroll
+#pragma unroll 2
   for (int blk = gw; blk < KB * GB; blk += 4) {
     const int n = (blk % KB) * 8 + n_lo;  // key within the chunk
     const int dblk = blk / KB;            // 64-column block
@@ -255,17 +269,17 @@ __device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, i
   }
   int issued = 0;
   if (gtid == 0) {
-    for (; issued < min(kRawStages, nchunk); ++issued)
+    for (; issued < min(S::kRawStages, nchunk); ++issued)
       issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + issued * S::RAW, &raw_full[issued],
                               &raw_ok[issued], status, ids);
   }
   int c = 0;
   for (; c < nchunk; ++c) {
-    const int st = c % kRawStages;
-    bool ok = wait_bar(&raw_full[st], (uint32_t)((c / kRawStages) & 1), misc, status);
-    const int slot = c % kSlots;
-    if (ok && c >= kSlots)
-      ok = wait_bar(&empty[slot], (uint32_t)((c / kSlots - 1) & 1), misc, status);
+    const int st = c % S::kRawStages;
+    bool ok = wait_bar(&raw_full[st], (uint32_t)((c / S::kRawStages) & 1), misc, status, true);
+    const int slot = c % S::kSlots;
+    if (ok && c >= S::kSlots)
+      ok = wait_bar(&empty[slot], (uint32_t)((c / S::kSlots - 1) & 1), misc, status, true);
     if (!ok) stop[c & 1] = 1;  // (the block is aborting: this chunk's data no longer matter)
     dequant_chunk<D, BS, FMT>(smem_u32(raw + st * S::RAW), raw_ok[st],
                               smem_u32(tiles + slot * S::TILE), c * S::kChunk, kv_end, gtid);
@@ -282,9 +296,9 @@ __device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, i
   // copies issued but never consumed (stopped early) must land before exit
   if (gtid == 0) {
     for (int k = c; k < issued; ++k) {
-      const int st = k % kRawStages;
+      const int st = k % S::kRawStages;
       for (int i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(&raw_full[st], (uint32_t)((k / kRawStages) & 1))) break;
+        if (mbar_try_wait(&raw_full[st], (uint32_t)((k / S::kRawStages) & 1))) break;
     }
   }
 }
@@ -320,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
 
   if (tid == 0) {
     for (int i = 0; i < S::kNumBars; ++i) {
-      const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kSlots) ||
-                        (i >= kBarPFull && i < kBarPFull + kSBufs) || i == kBarQReady;
+      const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) ||
+                        (i >= kBarPFull && i < kBarPFull + kMaxSBufs) || i == kBarQReady;
       mbar_init(&bars[i], many ? 128u : 1u);
     }
     misc->abort = 0;
@@ -385,31 +399,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     int done_chunks = 0;
     constexpr int CH = S::kChunk;
     for (int c = 0; c < nchunk; ++c) {
-      const int sb = c % kSBufs;
-      const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / kSBufs) & 1), misc, status);
+      const int sb = c % S::kSBufs;
+      const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / S::kSBufs) & 1), misc, status);
       if (!ok) stop[c & 1] = 1;
       tc::named_sync(kBarSoftmax, 128);
       if (stop[c & 1]) break;
       tc::fence_after_sync();
-      const uint32_t scol = S::kColS + CH * sb;
-      // logits of this chunk (s0: keys 0..31, s1: keys 32..63 when the chunk has 64)
-      uint32_t s0[32], s1[32];
-      tc::tmem_ld32(tb + lane_off + scol, s0);
-      if constexpr (CH == 64) tc::tmem_ld32(tb + lane_off + scol + 32, s1);
-      tc::tmem_wait_ld();
+      const uint32_t scol = tb + lane_off + S::kColS + CH * sb;
       const int key0 = c * CH;
       const int lim = min(pos + 1, kv_end) - key0;  // keys [key0, key0 + lim) are visible
-      // logits in log2 units, masked in place
+      // pass 1: max of the visible logits, in log2 units (32 columns at a time;
+      // the loops stay rolled to keep the hot code small)
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // (independent chains)
+#pragma unroll 1
+      for (int half = 0; half < CH / 32; ++half) {
+        uint32_t sv[32];
+        tc::tmem_ld32(scol + 32 * half, sv);
+        tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float x0 = (i < lim) ? __uint_as_float(s0[i]) * qmult : -INFINITY;
-        s0[i] = __float_as_uint(x0);
-        mx4[i & 3] = fmaxf(mx4[i & 3], x0);
-        if constexpr (CH == 64) {
-          const float x1 = (32 + i < lim) ? __uint_as_float(s1[i]) * qmult : -INFINITY;
-          s1[i] = __float_as_uint(x1);
-          mx4[i & 3] = fmaxf(mx4[i & 3], x1);
+        for (int i = 0; i < 32; ++i) {
+          const float x = (32 * half + i < lim) ? __uint_as_float(sv[i]) * qmult : -INFINITY;
+          mx4[i & 3] = fmaxf(mx4[i & 3], x);
         }
       }
       const float cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -427,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         // every PV MMA so far must be done before O is read and rewritten
         // (P-free of chunk c - 1: PV_{c-1} and, in issue order, every PV before it
         // done; that barrier is at most one phase behind here)
-        bool wok = wait_bar(&bars[kBarPFree + (c - 1) % kSBufs], (uint32_t)(((c - 1) / kSBufs) & 1),
+        bool wok = wait_bar(&bars[kBarPFree + (c - 1) % S::kSBufs], (uint32_t)(((c - 1) / S::kSBufs) & 1),
                             misc, status);
         if (__all_sync(0xffffffffu, wok)) {
           tc::fence_after_sync();
@@ -445,25 +455,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
           stop[(c + 1) & 1] = 1;  // read after the next chunk's barrier
         }
       }
-      // P = exp2(x - m) as f16 hi (columns scol .. scol + CH/2 - 1, keys in pairs)
-      // and lo = f16(P - hi) (the next CH/2 columns), 16 columns at a time
-      const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // all x are -inf then: P = 0
+      // pass 2: P = exp2(q.k * scale - m) per 16-key group, as f16 hi (8
+      // columns, keys in pairs) and lo = f16(P - hi) (the next 8), written over
+      // the group's own 16 logit columns (already read)
+      const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // no visible key yet: P = 0
       float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+      for (int grp = 0; grp < CH / 16; ++grp) {
+        uint32_t sv[16], pw[16];
+        tc::tmem_ld16(scol + 16 * grp, sv);
+        tc::tmem_wait_ld();
 #pragma unroll
-      for (int part = 0; part < CH / 32; ++part) {
-        const uint32_t(&xs)[32] = part ? s1 : s0;
-        uint32_t hw[16], lw[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(__uint_as_float(xs[2 * i]) - mu);
-          const float p1 = ex2(__uint_as_float(xs[2 * i + 1]) - mu);
+        for (int i = 0; i < 8; ++i) {
+          const int k0 = 16 * grp + 2 * i;
+          const float p0 = (k0 < lim) ? ex2(fmaf(__uint_as_float(sv[2 * i]), qmult, -mu)) : 0.0f;
+          const float p1 =
+              (k0 + 1 < lim) ? ex2(fmaf(__uint_as_float(sv[2 * i + 1]), qmult, -mu)) : 0.0f;
           ps4[i & 3] += p0 + p1;
-          hw[i] = pack_f16x2(p0, p1);
-          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
-          lw[i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
+          pw[i] = pack_f16x2(p0, p1);
+          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
+          pw[8 + i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
         }
-        tc::tmem_st16(tb + lane_off + scol + 16 * part, hw);
-        tc::tmem_st16(tb + lane_off + scol + CH / 2 + 16 * part, lw);
+        tc::tmem_st16(scol + 16 * grp, pw);
       }
       l_run += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
       tc::tmem_wait_st();
@@ -562,47 +575,60 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
       const uint32_t kbase = smem_u32(base + S::kOffK), vbase = smem_u32(base + S::kOffV);
       bool ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
-      // S = Q K^T of chunk j into TMEM buffer j % 4 (after the PV MMAs that read
-      // the P held there, chunk j - 4, have completed)
+      constexpr int NB = S::kSBufs, NS = S::kSlots;
+      // S = Q K^T of chunk j into TMEM buffer j % NB (after the PV MMAs that
+      // read the P held there, chunk j - NB, have completed)
       auto issue_s = [&](int j) -> bool {
-        const int sb = j % kSBufs, slot = j % kSlots;
-        bool k = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / kSlots) & 1), misc, status);
-        if (k && j >= kSBufs)
-          k = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / kSBufs - 1) & 1), misc, status);
+        const int sb = j % NB, slot = j % NS;
+        bool k = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1), misc, status);
+        if (k && j >= NB)
+          k = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1), misc, status);
         if (!k) return false;
         tc::fence_after_sync();
-        const uint32_t kt = kbase + slot * S::TILE;
+        const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
         const uint32_t dS = tb + S::kColS + CH * sb;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t desc =
-              tc::sw128_desc(kt + (kk >> 2) * (CH * 128) + (kk & 3) * 32, 16, 1024);
+          // start address advanced in 16-byte units (stays below 2^14 units)
+          const uint64_t desc = desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
           tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
         }
         tc::commit(&bars[kBarKEmpty + slot]);
         tc::commit(&bars[kBarSFull + sb]);
         return true;
       };
-      // order: S_0, S_1, then S_{c+2}, PV_c for c = 0, 1, ...: two S chunks are
-      // queued on the tensor core while the softmax of chunk c runs
-      for (int j = 0; ok && j < min(2, nchunk); ++j) ok = issue_s(j);
-      for (int c = 0; ok && c < nchunk; ++c) {
-        if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
-        const int pb = c % kSBufs, slot = c % kSlots;
-        ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / kSBufs) & 1), misc, status);
-        if (ok) ok = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / kSlots) & 1), misc, status);
-        if (!ok) break;
+      // O += P V of chunk c (P hi, then P lo, per 16 keys)
+      auto issue_pv = [&](int c) -> bool {
+        const int pb = c % NB, slot = c % NS;
+        bool k = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1), misc, status);
+        if (k) k = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1), misc, status);
+        if (!k) return false;
         tc::fence_after_sync();
-        const uint32_t vt = vbase + slot * S::TILE;
+        const uint64_t desc0 = tc::sw128_desc(vbase + slot * S::TILE, CH * 128, 1024);
         const uint32_t pS = tb + S::kColS + CH * pb;
 #pragma unroll
         for (int i = 0; i < CH / 16; ++i) {
-          const uint64_t desc = tc::sw128_desc(vt + i * 2048, CH * 128, 1024);
-          tc::mma_ts(tb + S::kColO, pS + i * 8, desc, kIdescPV, c > 0 || i > 0);
-          tc::mma_ts(tb + S::kColO, pS + CH / 2 + i * 8, desc, kIdescPV, true);
+          const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
+          tc::mma_ts(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
+          tc::mma_ts(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
         }
         tc::commit(&bars[kBarVEmpty + slot]);
         tc::commit(&bars[kBarPFree + pb]);
+        return true;
+      };
+      // S_0, S_1 first; then per chunk c, with four buffers S_{c+2} (its buffer
+      // was read by PV_{c-2}) before PV_c, so two S chunks are queued while the
+      // softmax of chunk c runs; with two buffers PV_c first, then S_{c+2} in
+      // the buffer PV_c has just read
+      for (int j = 0; ok && j < min(2, nchunk); ++j) ok = issue_s(j);
+      for (int c = 0; ok && c < nchunk; ++c) {
+        if constexpr (NB == 2) {
+          if (!(ok = issue_pv(c))) break;
+          if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
+        } else {
+          if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
+          if (!(ok = issue_pv(c))) break;
+        }
       }
       // every MMA issued has completed before TMEM is released
       tc::commit(&bars[kBarFin]);
@@ -610,10 +636,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         if (mbar_try_wait(&bars[kBarFin], 0u)) break;
     }
     __syncwarp();
-  } else if (tid < kVGroup0) {
-    kv_role<D, BS, FMT>(a, 0, b, h, nchunk, kv_end, base, bars, misc, status);
   } else {
-    kv_role<D, BS, FMT>(a, 1, b, h, nchunk, kv_end, base, bars, misc, status);
+    // K (warps 5-8) and V (warps 9-12) run one copy of the code
+    kv_role<D, BS, FMT>(a, tid >= kVGroup0 ? 1 : 0, b, h, nchunk, kv_end, base, bars, misc,
+                        status);
   }
 
   tc::fence_before_sync();
