@@ -16,21 +16,28 @@
 //                (f16, 128B-swizzled shared tile, K-major), D = S (fp32, TMEM)
 //   P  = exp2(S * scale - m) in fp32, split into f16 hi + lo (~22 bits: f16
 //        alone misses the 2e-3 bound on outlier-heavy rows), written back to
-//        TMEM over S's columns
+//        TMEM over S's columns: per 16 keys, 8 columns of hi then 8 of lo
 //   O += P V     A = P hi, then P lo (TMEM), B = V chunk (the same swizzled
 //                tile layout read MN-major), D = O (fp32, TMEM)
+// S/P buffers in TMEM: four (two at head size 256, where O and Q take 384 of
+// the 512 columns), so S of later chunks is computed while the softmax of
+// chunk c runs.
 // E2M1 * E4M3 has at most 6 significant bits in [2^-10, 2688], so K and V are
 // exact in f16; k_scale is folded into the logit scale and v_scale into the
 // output. Q is scaled per row by a power of two putting max |q| in
 // [2^14, 2^15), where f16 keeps every bf16 bit. The running max moves only when
 // a chunk's max exceeds it by more than 2^8 (then O is rescaled in TMEM).
 //
-// Warp roles (13 warps):
+// Warp roles (16 warps):
 //   0-3   Q rows into TMEM, softmax (thread i = row i = TMEM lane i), epilogue
-//   4     TMEM allocation; one thread issues every MMA and commit
-//   5-8   K pages: bulk copies of a chunk's NVFP4 pages into a 3-stage ring,
-//         then dequantization into one of two f16 K tiles
-//   9-12  V pages: the same for V
+//   4     TMEM allocation; one thread issues the PV MMAs
+//   5-8   K: dequantization of a chunk's raw NVFP4 pages into an f16 tile slot
+//   9-12  V: the same for V (one code copy with K)
+//   13    one thread issues the S MMAs
+//   14-15 one thread each issues the bulk copies of K (V) pages into a raw
+//         stage ring
+// The hot loops are kept rolled where unrolling buys little: with every role
+// resident at once, an unrolled kernel outgrows the instruction cache.
 // Every mbarrier wait is bounded; a wait that gives up raises NVFP4_DEV_TIMEOUT
 // and makes the whole block stop, wait for its copies and MMAs, free its TMEM
 // and return.
@@ -50,14 +57,28 @@ constexpr int kMaxRawStages = 3;  // raw page stages per K and V (at most)
 // block ids of a CTA's pages held in shared memory (longer ranges read them
 // from the block table as they go)
 constexpr int kMaxIds = 4096;
-constexpr int kThreads = 13 * 32;
-constexpr int kMmaWarp = 4;
+constexpr int kThreads = 16 * 32;
+constexpr int kMmaWarp = 4;    // TMEM allocation, PV MMAs
+constexpr int kSWarp = 13;     // S MMAs
+constexpr int kCopyWarp0 = 14; // K page copies (warp 15: V)
 constexpr int kKGroup0 = 5 * 32;  // first thread of the K warps
 constexpr int kVGroup0 = 9 * 32;  // first thread of the V warps
-constexpr uint32_t kBarK = 1, kBarV = 2, kBarSoftmax = 3;  // named barriers (128 threads)
+constexpr uint32_t kBarSoftmax = 3, kBarCopy = 4;  // named barriers (128, 64 threads)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;
 constexpr int kMaxPolls = 1 << 22;
+#ifndef PREFILL_SUSPEND_NS
+#define PREFILL_SUSPEND_NS 1000
+#endif
+#ifndef KV_WAIT
+#define KV_WAIT kWaitSleep
+#endif
+#ifndef MMA_WAIT
+#define MMA_WAIT kWaitSpin
+#endif
+#ifndef SM_WAIT
+#define SM_WAIT kWaitSpin
+#endif
 // a CTA keeps the SM to itself (its TMEM allocation is the whole SM's)
 constexpr size_t kMinSmem = 120 * 1024;
 
@@ -73,7 +94,8 @@ enum : int {
   kBarPFull = kBarSFull + kMaxSBufs, // [4] P chunk in TMEM (128 arrivals)
   kBarPFree = kBarPFull + kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
   kBarQReady = kBarPFree + kMaxSBufs,  // Q rows in TMEM (128 arrivals)
-  kBarFin = kBarQReady + 1,       // every MMA issued done (commit)
+  kBarRawEmpty = kBarQReady + 1,  // [2][3] K, V raw stage read by every dequant thread (128 arrivals)
+  kBarFin = kBarRawEmpty + 2 * kMaxRawStages,  // every MMA issued done (2 commits)
   kNumBarriers = kBarFin + 1
 };
 
@@ -104,8 +126,8 @@ struct PrefillShape {
   static constexpr int kOffBar = kOffVraw + kRawStages * RAW;
   static constexpr int kNumBars = kNumBarriers;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kOffIds = kOffMisc + 64;             // [2][kMaxIds] block ids (K, V)
-  static constexpr int kBytes = kOffIds + 2 * kMaxIds * 4;
+  static constexpr int kOffIds = kOffMisc + 64;             // [kMaxIds] block ids
+  static constexpr int kBytes = kOffIds + kMaxIds * 4;
   static size_t smem_bytes() {
     const size_t need = (size_t)kBytes + 1024;  // + alignment of the base
     return need > kMinSmem ? need : kMinSmem;
@@ -123,25 +145,41 @@ struct PrefillShape {
 struct Misc {
   uint32_t tmem_base;
   int abort;  // a wait of some role gave up: everyone stops
-  // per role group (K, V, softmax), two alternating slots: chunk c's stop flag
-  // is written before the group's barrier of chunk c and read after it; the
-  // slot is written again only at chunk c + 2, after every thread of the group
-  // has passed the barrier of chunk c + 1
-  int group_stop[3][2];
+  // the softmax group's stop flag, two alternating slots: chunk c's flag is
+  // written before the group's barrier of chunk c and read after it; the slot
+  // is written again only at chunk c + 2, after every thread of the group has
+  // passed the barrier of chunk c + 1
+  int softmax_stop[2];
   uint32_t raw_ok[2][kMaxRawStages];  // per raw stage: bit i = page i of the chunk was copied
 };
 
 // Bounded wait that also gives up once another role has aborted the block.
-// A waiter off the critical path (relaxed) sleeps briefly between polls, so
-// that it leaves the issue slots of its SM sub-partition to the softmax and
-// MMA warps there.
+// Waiters share their SM sub-partition's issue slots with the warps doing the
+// work they wait for, so they do not spin flat out: kWaitSuspend polls let the
+// hardware suspend the thread until the phase completes (or a time hint runs
+// out), kWaitSleep polls sleep briefly between tries.
+enum WaitMode { kWaitSpin = 0, kWaitSleep = 1, kWaitSuspend = 2 };
 constexpr unsigned kRelaxedSleepNs = 64;
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(PREFILL_SUSPEND_NS)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* misc,
-                                         uint32_t* status, bool relaxed = false) {
+                                         uint32_t* status, int mode = kWaitSpin) {
   for (int i = 0; i < kMaxPolls; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mode == kWaitSuspend ? mbar_try_wait_suspend(bar, parity) : mbar_try_wait(bar, parity))
+      return true;
     if ((i & 127) == 127 && *reinterpret_cast<volatile int*>(&misc->abort)) return false;
-    if (relaxed) __nanosleep(kRelaxedSleepNs);
+    if (mode == kWaitSleep) __nanosleep(kRelaxedSleepNs);
   }
   atomicOr(status, kDevTimeout);
   *reinterpret_cast<volatile int*>(&misc->abort) = 1;
@@ -183,123 +221,173 @@ __device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h
 }
 
 // Dequantize one chunk from its raw stage into an f16 tile laid out for the
-// MMA: 64-column blocks of [chunk keys][64 d] f16, 128-byte rows, the 16-byte
+// MMA: 64-column blocks of [64 keys][64 d] f16, 128-byte rows, the 16-byte
 // chunk j of row n stored at chunk j ^ (n % 8). A thread converts one scale
-// group (16 elements of one key: 8 code bytes and their E4M3 scale) per step;
-// a warp step covers 8 keys x 4 groups, so both the code loads and the tile
-// stores are free of bank conflicts. Keys at or past kv_end, and keys of pages
-// not copied, become zeros. 128 threads.
+// group (16 elements of one key: 8 code bytes and their E4M3 scale) per step:
+// warp w, lane l takes keys 8 (w + 4 j) + l % 8 (j = 0, 1) and group l / 8 of
+// every 64-column block, so a warp step covers 8 keys x 4 groups and both the
+// code loads and the tile stores are free of bank conflicts. Keys at or past
+// the visible end, and keys of pages not copied, become zeros. 128 threads.
+//
+// The thread's offsets are the same for every chunk: computed once.
+struct DequantPlan {
+  uint32_t row[2];   // byte offset of key j's row in a raw stage
+  uint32_t dst[2];   // byte offset of key j's 128-byte row in a tile's first 64-column block
+  uint32_t sw0, sw1; // swizzled offsets of the thread's two 16-byte chunks in a row
+  uint32_t goff;     // 8 x (group within a 64-column block)
+  int n[2];          // the keys, within the chunk
+  int pg[2];         // their pages, within the chunk
+};
+
 template <int D, int BS, int FMT>
-__device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_t tile, int key0,
-                                              int kv_end, int gtid) {
+__device__ __forceinline__ DequantPlan dequant_plan(int gtid) {
   using S = PrefillShape<D, BS, FMT>;
-  constexpr int KB = S::kChunk / 8;  // blocks of 8 keys
-  constexpr int GB = D / 64;         // blocks of 4 groups (one 64-column tile block each)
+  static_assert(S::kChunk == 64, "the plan covers 64-key chunks with 4 warps");
   const int lane = gtid & 31, gw = gtid >> 5;
   const int n_lo = lane & 7, g_lo = lane >> 3;
-#pragma unroll 2
-  for (int blk = gw; blk < KB * GB; blk += 4) {
-    const int n = (blk % KB) * 8 + n_lo;  // key within the chunk
-    const int dblk = blk / KB;            // 64-column block
-    const int g = dblk * 4 + g_lo;        // scale group of the row
-    const bool valid = (key0 + n < kv_end) && ((ok >> (n / BS)) & 1u);
-    const uint32_t row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
-    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-    if (valid) {
-      if constexpr (FMT) {  // FP8 row: 16 E4M3 bytes -> 16 f16 (exact)
-        uint32_t w[4];
-        lds_v4(row + 16 * g, w);
-        lo.x = e4m3x2_to_f16x2(w[0] & 0xFFFFu);
-        lo.y = e4m3x2_to_f16x2(w[0] >> 16);
-        lo.z = e4m3x2_to_f16x2(w[1] & 0xFFFFu);
-        lo.w = e4m3x2_to_f16x2(w[1] >> 16);
-        hi.x = e4m3x2_to_f16x2(w[2] & 0xFFFFu);
-        hi.y = e4m3x2_to_f16x2(w[2] >> 16);
-        hi.z = e4m3x2_to_f16x2(w[3] & 0xFFFFu);
-        hi.w = e4m3x2_to_f16x2(w[3] >> 16);
-      } else {  // NVFP4 row: 8 code bytes x one E4M3 scale -> 16 f16 (exact)
-        uint32_t c0, c1;
-        if constexpr (S::F % 8 == 0) {
-          lds_v2(row + 8 * g, c0, c1);
-        } else {
-          c0 = ld_shared_u32(row + 8 * g);
-          c1 = ld_shared_u32(row + 8 * g + 4);
+  DequantPlan pl;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int n = (gw + 4 * j) * 8 + n_lo;
+    pl.n[j] = n;
+    pl.pg[j] = n / BS;
+    pl.row[j] = (uint32_t)((n / BS) * S::PAGE + (n % BS) * S::F);
+    pl.dst[j] = (uint32_t)(n * 128);
+  }
+  pl.sw0 = (uint32_t)(((2 * g_lo) ^ n_lo) << 4);
+  pl.sw1 = (uint32_t)(((2 * g_lo + 1) ^ n_lo) << 4);
+  pl.goff = (uint32_t)(8 * g_lo);
+  return pl;
+}
+
+template <int D, int BS, int FMT>
+__device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_t tile, int lim,
+                                              const DequantPlan& pl) {
+  using S = PrefillShape<D, BS, FMT>;
+  bool valid[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) valid[j] = (pl.n[j] < lim) && ((ok >> pl.pg[j]) & 1u);
+#pragma unroll
+  for (int dblk = 0; dblk < D / 64; ++dblk) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t row = raw + pl.row[j];
+      // (loaded and converted whatever valid says: the stage's bytes exist,
+      // stale for a key not copied, and the result is zeroed after)
+      uint4 lo, hi;
+      {
+        if constexpr (FMT) {  // FP8 row: 16 E4M3 bytes -> 16 f16 (exact)
+          uint32_t w[4];
+          lds_v4(row + 64 * dblk + 2 * pl.goff, w);
+          lo.x = e4m3x2_to_f16x2(w[0] & 0xFFFFu);
+          lo.y = e4m3x2_to_f16x2(w[0] >> 16);
+          lo.z = e4m3x2_to_f16x2(w[1] & 0xFFFFu);
+          lo.w = e4m3x2_to_f16x2(w[1] >> 16);
+          hi.x = e4m3x2_to_f16x2(w[2] & 0xFFFFu);
+          hi.y = e4m3x2_to_f16x2(w[2] >> 16);
+          hi.z = e4m3x2_to_f16x2(w[3] & 0xFFFFu);
+          hi.w = e4m3x2_to_f16x2(w[3] >> 16);
+        } else {  // NVFP4 row: 8 code bytes x one E4M3 scale -> 16 f16 (exact)
+          const uint32_t ca = row + 32 * dblk + pl.goff;
+          uint32_t c0, c1;
+          if constexpr (S::F % 8 == 0) {
+            lds_v2(ca, c0, c1);
+          } else {
+            c0 = ld_shared_u32(ca);
+            c1 = ld_shared_u32(ca + 4);
+          }
+          const uint32_t sb = lds_b8(row + D / 2 + 4 * dblk + (pl.goff >> 3));
+          const uint32_t s2 = e4m3x2_to_f16x2(sb * 0x101u);
+          uint32_t x[4], y[4];
+          e2m1x8_to_f16x2x4(c0, x);
+          e2m1x8_to_f16x2x4(c1, y);
+          lo = make_uint4(hmul2_u32(x[0], s2), hmul2_u32(x[1], s2), hmul2_u32(x[2], s2),
+                          hmul2_u32(x[3], s2));
+          hi = make_uint4(hmul2_u32(y[0], s2), hmul2_u32(y[1], s2), hmul2_u32(y[2], s2),
+                          hmul2_u32(y[3], s2));
         }
-        const uint32_t sb = lds_b8(row + D / 2 + g);
-        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
-        uint32_t x[4], y[4];
-        e2m1x8_to_f16x2x4(c0, x);
-        e2m1x8_to_f16x2x4(c1, y);
-        lo = make_uint4(hmul2_u32(x[0], s2), hmul2_u32(x[1], s2), hmul2_u32(x[2], s2),
-                        hmul2_u32(x[3], s2));
-        hi = make_uint4(hmul2_u32(y[0], s2), hmul2_u32(y[1], s2), hmul2_u32(y[2], s2),
-                        hmul2_u32(y[3], s2));
       }
+      if (!valid[j]) lo = hi = make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t dst = tile + dblk * (S::kChunk * 128) + pl.dst[j];
+      sts_v4(dst + pl.sw0, lo);
+      sts_v4(dst + pl.sw1, hi);
     }
-    const uint32_t dst = tile + dblk * (S::kChunk * 128) + n * 128;
-    const int c = 2 * g_lo;  // 16-byte chunks c, c + 1 of the 128-byte row
-    sts_v4(dst + ((c ^ (n & 7)) << 4), lo);
-    sts_v4(dst + (((c + 1) ^ (n & 7)) << 4), hi);
   }
 }
 
-// The copy + dequant pipeline of one of K (kv = 0) and V (kv = 1).
+// Dequantization of one of K (kv = 0) and V (kv = 1), 128 threads: per chunk,
+// wait for its raw pages and a free tile slot, convert, and release both.
+// Every warp runs at its own pace (no barrier among the four).
 template <int D, int BS, int FMT>
-__device__ __forceinline__ void kv_role(const AttentionArgs& a, int kv, int b, int h, int nchunk,
-                                        int kv_end, uint8_t* base, uint64_t* bars, Misc* misc,
-                                        uint32_t* status) {
+__device__ __forceinline__ void dequant_role(int kv, int nchunk, int kv_end, uint8_t* base,
+                                             uint64_t* bars, Misc* misc, uint32_t* status) {
   using S = PrefillShape<D, BS, FMT>;
   const int gtid = threadIdx.x - (kv ? kVGroup0 : kKGroup0);
-  const uint32_t bar_id = kv ? kBarV : kBarK;
-  uint8_t* raw = base + (kv ? S::kOffVraw : S::kOffKraw);
-  uint8_t* tiles = base + (kv ? S::kOffV : S::kOffK);
+  const uint32_t raw_s = smem_u32(base + (kv ? S::kOffVraw : S::kOffKraw));
+  const uint32_t tiles_s = smem_u32(base + (kv ? S::kOffV : S::kOffK));
   uint64_t* raw_full = bars + (kv ? kBarVraw : kBarKraw);
+  uint64_t* raw_empty = bars + kBarRawEmpty + kv * kMaxRawStages;
   uint64_t* full = bars + (kv ? kBarVFull : kBarKFull);
   uint64_t* empty = bars + (kv ? kBarVEmpty : kBarKEmpty);
+  const volatile uint32_t* raw_ok = misc->raw_ok[kv];
+  const DequantPlan plan = dequant_plan<D, BS, FMT>(gtid);
+  for (int c = 0; c < nchunk; ++c) {
+    const int st = c % S::kRawStages, slot = c % S::kSlots;
+    bool ok = wait_bar(&raw_full[st], (uint32_t)((c / S::kRawStages) & 1), misc, status, KV_WAIT);
+    if (ok && c >= S::kSlots)
+      ok = wait_bar(&empty[slot], (uint32_t)((c / S::kSlots - 1) & 1), misc, status, KV_WAIT);
+    if (!ok) break;  // the block is aborting
+    dequant_chunk<D, BS, FMT>(raw_s + st * S::RAW, raw_ok[st], tiles_s + slot * S::TILE,
+                              kv_end - c * S::kChunk, plan);
+    // generic-proxy writes of the tile (read by the tensor core) and reads of
+    // the raw stage (next written by a bulk copy), both before the arrivals
+    fence_proxy_async_smem();
+    tc::mbar_arrive(&full[slot]);
+    tc::mbar_arrive(&raw_empty[st]);
+  }
+}
+
+// Page copies of one of K (kv = 0) and V (kv = 1), one thread: chunk c goes
+// into raw stage c % kRawStages once every dequant thread has released the
+// chunk that stage held. Both copy warps first stage the CTA's block ids in
+// shared memory (K and V pages share them). Before exit the thread waits for
+// every copy it issued to land (the copies write this CTA's shared memory).
+template <int D, int BS, int FMT>
+__device__ __forceinline__ void copy_role(const AttentionArgs& a, int kv, int b, int h, int nchunk,
+                                          int kv_end, uint8_t* base, uint64_t* bars, Misc* misc,
+                                          uint32_t* status) {
+  using S = PrefillShape<D, BS, FMT>;
+  const int lane = threadIdx.x & 31;
+  uint8_t* raw = base + (kv ? S::kOffVraw : S::kOffKraw);
+  uint64_t* raw_full = bars + (kv ? kBarVraw : kBarKraw);
+  uint64_t* raw_empty = bars + kBarRawEmpty + kv * kMaxRawStages;
   uint32_t* raw_ok = misc->raw_ok[kv];
-  volatile int* stop = misc->group_stop[kv];
-  // the block ids of this CTA's pages, loaded once (coalesced) into shared memory
   const int npages = min((kv_end + BS - 1) / BS, a.max_blocks_per_seq);
   int* ids = nullptr;
   if (npages <= kMaxIds) {
-    ids = reinterpret_cast<int*>(base + S::kOffIds) + kv * kMaxIds;
+    ids = reinterpret_cast<int*>(base + S::kOffIds);
     const int* row = a.block_table + (long long)b * a.max_blocks_per_seq;
-    for (int p = gtid; p < npages; p += 128) ids[p] = __ldg(row + p);
-    tc::named_sync(bar_id, 128);
+    for (int p = kv * 32 + lane; p < npages; p += 64) ids[p] = __ldg(row + p);
+    tc::named_sync(kBarCopy, 64);
   }
+  if (lane != 0) return;
   int issued = 0;
-  if (gtid == 0) {
-    for (; issued < min(S::kRawStages, nchunk); ++issued)
-      issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + issued * S::RAW, &raw_full[issued],
-                              &raw_ok[issued], status, ids);
-  }
-  int c = 0;
-  for (; c < nchunk; ++c) {
+  for (int c = 0; c < nchunk; ++c) {
     const int st = c % S::kRawStages;
-    bool ok = wait_bar(&raw_full[st], (uint32_t)((c / S::kRawStages) & 1), misc, status, true);
-    const int slot = c % S::kSlots;
-    if (ok && c >= S::kSlots)
-      ok = wait_bar(&empty[slot], (uint32_t)((c / S::kSlots - 1) & 1), misc, status, true);
-    if (!ok) stop[c & 1] = 1;  // (the block is aborting: this chunk's data no longer matter)
-    dequant_chunk<D, BS, FMT>(smem_u32(raw + st * S::RAW), raw_ok[st],
-                              smem_u32(tiles + slot * S::TILE), c * S::kChunk, kv_end, gtid);
-    fence_proxy_async_smem();  // generic writes -> read by the tensor core
-    tc::mbar_arrive(&full[slot]);
-    tc::named_sync(bar_id, 128);  // every thread is done with raw stage st
-    if (stop[c & 1]) break;  // (the drain below also covers chunk c's copies)
-    if (gtid == 0 && issued < nchunk) {
-      issue_chunk<D, BS, FMT>(a, b, h, kv, issued, kv_end, raw + st * S::RAW, &raw_full[st],
-                              &raw_ok[st], status, ids);
-      ++issued;
-    }
+    if (c >= S::kRawStages &&
+        !wait_bar(&raw_empty[st], (uint32_t)((c / S::kRawStages - 1) & 1), misc, status,
+                  kWaitSleep))
+      break;
+    issue_chunk<D, BS, FMT>(a, b, h, kv, c, kv_end, raw + st * S::RAW, &raw_full[st], &raw_ok[st],
+                            status, ids);
+    issued = c + 1;
   }
-  // copies issued but never consumed (stopped early) must land before exit
-  if (gtid == 0) {
-    for (int k = c; k < issued; ++k) {
-      const int st = k % S::kRawStages;
-      for (int i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(&raw_full[st], (uint32_t)((k / S::kRawStages) & 1))) break;
-    }
+  // the last copy of each stage (earlier ones were consumed before the stage
+  // was refilled) has landed
+  for (int k = max(0, issued - S::kRawStages); k < issued; ++k) {
+    const int st = k % S::kRawStages;
+    for (int i = 0; i < kMaxPolls; ++i)
+      if (mbar_try_wait(&raw_full[st], (uint32_t)((k / S::kRawStages) & 1))) break;
   }
 }
 
@@ -335,11 +423,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
   if (tid == 0) {
     for (int i = 0; i < S::kNumBars; ++i) {
       const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) ||
-                        (i >= kBarPFull && i < kBarPFull + kMaxSBufs) || i == kBarQReady;
-      mbar_init(&bars[i], many ? 128u : 1u);
+                        (i >= kBarPFull && i < kBarPFull + kMaxSBufs) || i == kBarQReady ||
+                        (i >= kBarRawEmpty && i < kBarRawEmpty + 2 * kMaxRawStages);
+      mbar_init(&bars[i], many ? 128u : (i == kBarFin ? 2u : 1u));
     }
     misc->abort = 0;
-    for (int i = 0; i < 3; ++i) misc->group_stop[i][0] = misc->group_stop[i][1] = 0;
+    misc->softmax_stop[0] = misc->softmax_stop[1] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tc::tmem_alloc(&misc->tmem_base, S::kTmemCols);
@@ -395,12 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     tc::mbar_arrive(&bars[kBarQReady]);
 
     float m_run = -INFINITY, l_run = 0.0f;
-    volatile int* stop = misc->group_stop[2];
+    volatile int* stop = misc->softmax_stop;
     int done_chunks = 0;
     constexpr int CH = S::kChunk;
     for (int c = 0; c < nchunk; ++c) {
       const int sb = c % S::kSBufs;
-      const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / S::kSBufs) & 1), misc, status);
+      const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / S::kSBufs) & 1), misc, status, SM_WAIT);
       if (!ok) stop[c & 1] = 1;
       tc::named_sync(kBarSoftmax, 128);
       if (stop[c & 1]) break;
@@ -567,79 +656,76 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       }  // row_ok
       __syncwarp();
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------ MMA issue (one thread)
+  } else if (warp == kMmaWarp || warp == kSWarp) {
+    // ------------------------------------------------ MMA issue: one thread of
+    // warp kSWarp issues every S = Q K^T, one thread of warp kMmaWarp every
+    // O += P V; each commits its own barriers (a commit tracks the MMAs its
+    // thread issued), and the two order through them: S_j is issued once PV_{j-NB}
+    // (which read the P buffer S_j overwrites) has completed, PV_c once the
+    // softmax has turned S_c into P_c.
     if (lane == 0 && nchunk > 0) {
       constexpr int CH = S::kChunk;
-      constexpr uint32_t kIdescS = tc::idesc_f16(kRows, CH, false);
-      constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
-      const uint32_t kbase = smem_u32(base + S::kOffK), vbase = smem_u32(base + S::kOffV);
-      bool ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
       constexpr int NB = S::kSBufs, NS = S::kSlots;
-      // S = Q K^T of chunk j into TMEM buffer j % NB (after the PV MMAs that
-      // read the P held there, chunk j - NB, have completed)
-      auto issue_s = [&](int j) -> bool {
-        const int sb = j % NB, slot = j % NS;
-        bool k = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1), misc, status);
-        if (k && j >= NB)
-          k = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1), misc, status);
-        if (!k) return false;
-        tc::fence_after_sync();
-        const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
-        const uint32_t dS = tb + S::kColS + CH * sb;
+      bool ok = true;
+      if (warp == kSWarp) {
+        constexpr uint32_t kIdescS = tc::idesc_f16(kRows, CH, false);
+        const uint32_t kbase = smem_u32(base + S::kOffK);
+        ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
+        for (int j = 0; ok && j < nchunk; ++j) {
+          const int sb = j % NB, slot = j % NS;
+          ok = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1), misc, status, MMA_WAIT);
+          if (ok && j >= NB)
+            ok = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1), misc, status, MMA_WAIT);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
+          const uint32_t dS = tb + S::kColS + CH * sb;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // start address advanced in 16-byte units (stays below 2^14 units)
-          const uint64_t desc = desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
-          tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // start address advanced in 16-byte units (stays below 2^14 units)
+            const uint64_t desc =
+                desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
+            tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+          }
+          tc::commit(&bars[kBarKEmpty + slot]);
+          tc::commit(&bars[kBarSFull + sb]);
         }
-        tc::commit(&bars[kBarKEmpty + slot]);
-        tc::commit(&bars[kBarSFull + sb]);
-        return true;
-      };
-      // O += P V of chunk c (P hi, then P lo, per 16 keys)
-      auto issue_pv = [&](int c) -> bool {
-        const int pb = c % NB, slot = c % NS;
-        bool k = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1), misc, status);
-        if (k) k = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1), misc, status);
-        if (!k) return false;
-        tc::fence_after_sync();
-        const uint64_t desc0 = tc::sw128_desc(vbase + slot * S::TILE, CH * 128, 1024);
-        const uint32_t pS = tb + S::kColS + CH * pb;
+      } else {
+        constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
+        const uint32_t vbase = smem_u32(base + S::kOffV);
+        for (int c = 0; ok && c < nchunk; ++c) {
+          const int pb = c % NB, slot = c % NS;
+          ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1), misc, status, MMA_WAIT);
+          if (ok) ok = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1), misc, status, MMA_WAIT);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint64_t desc0 = tc::sw128_desc(vbase + slot * S::TILE, CH * 128, 1024);
+          const uint32_t pS = tb + S::kColS + CH * pb;
 #pragma unroll
-        for (int i = 0; i < CH / 16; ++i) {
-          const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
-          tc::mma_ts(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
-          tc::mma_ts(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
-        }
-        tc::commit(&bars[kBarVEmpty + slot]);
-        tc::commit(&bars[kBarPFree + pb]);
-        return true;
-      };
-      // S_0, S_1 first; then per chunk c, with four buffers S_{c+2} (its buffer
-      // was read by PV_{c-2}) before PV_c, so two S chunks are queued while the
-      // softmax of chunk c runs; with two buffers PV_c first, then S_{c+2} in
-      // the buffer PV_c has just read
-      for (int j = 0; ok && j < min(2, nchunk); ++j) ok = issue_s(j);
-      for (int c = 0; ok && c < nchunk; ++c) {
-        if constexpr (NB == 2) {
-          if (!(ok = issue_pv(c))) break;
-          if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
-        } else {
-          if (c + 2 < nchunk && !(ok = issue_s(c + 2))) break;
-          if (!(ok = issue_pv(c))) break;
+          for (int i = 0; i < CH / 16; ++i) {  // P hi, then P lo, per 16 keys
+            const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
+            tc::mma_ts(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
+            tc::mma_ts(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
+          }
+          tc::commit(&bars[kBarVEmpty + slot]);
+          tc::commit(&bars[kBarPFree + pb]);
         }
       }
-      // every MMA issued has completed before TMEM is released
+      // every MMA this thread issued has completed: the final barrier counts
+      // both issuers
       tc::commit(&bars[kBarFin]);
+    }
+    if (warp == kMmaWarp && lane == 0 && nchunk > 0) {
+      // (TMEM is released by this warp below, after every MMA has completed)
       for (int i = 0; i < kMaxPolls; ++i)
         if (mbar_try_wait(&bars[kBarFin], 0u)) break;
     }
     __syncwarp();
+  } else if (warp >= kCopyWarp0) {
+    copy_role<D, BS, FMT>(a, warp - kCopyWarp0, b, h, nchunk, kv_end, base, bars, misc, status);
   } else {
     // K (warps 5-8) and V (warps 9-12) run one copy of the code
-    kv_role<D, BS, FMT>(a, tid >= kVGroup0 ? 1 : 0, b, h, nchunk, kv_end, base, bars, misc,
-                        status);
+    dequant_role<D, BS, FMT>(tid >= kVGroup0 ? 1 : 0, nchunk, kv_end, base, bars, misc, status);
   }
 
   tc::fence_before_sync();
