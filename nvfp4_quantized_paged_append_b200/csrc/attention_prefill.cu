@@ -28,14 +28,16 @@
 // [2^14, 2^15), where f16 keeps every bf16 bit. The running max moves only when
 // a chunk's max exceeds it by more than 2^8 (then O is rescaled in TMEM).
 //
-// Warp roles (16 warps):
-//   0-3   Q rows into TMEM, softmax (thread i = row i = TMEM lane i), epilogue
+// Warp roles (20 warps):
+//   0-3   Q rows into TMEM; softmax of keys [0, 32) of each chunk and epilogue
+//         of O columns [0, D/2) (thread i = row i = TMEM lane i)
 //   4     TMEM allocation; one thread issues the PV MMAs
 //   5-8   K: dequantization of a chunk's raw NVFP4 pages into an f16 tile slot
 //   9-12  V: the same for V (one code copy with K)
 //   13    one thread issues the S MMAs
 //   14-15 one thread each issues the bulk copies of K (V) pages into a raw
 //         stage ring
+//   16-19 softmax of keys [32, 64) and epilogue of O columns [D/2, D)
 // The hot loops are kept rolled where unrolling buys little: with every role
 // resident at once, an unrolled kernel outgrows the instruction cache.
 // Every mbarrier wait is bounded; a wait that gives up raises NVFP4_DEV_TIMEOUT
@@ -57,13 +59,14 @@ constexpr int kMaxRawStages = 3;  // raw page stages per K and V (at most)
 // block ids of a CTA's pages held in shared memory (longer ranges read them
 // from the block table as they go)
 constexpr int kMaxIds = 4096;
-constexpr int kThreads = 16 * 32;
+constexpr int kThreads = 20 * 32;
 constexpr int kMmaWarp = 4;    // TMEM allocation, PV MMAs
 constexpr int kSWarp = 13;     // S MMAs
 constexpr int kCopyWarp0 = 14; // K page copies (warp 15: V)
+constexpr int kSoftmax1Warp0 = 16;  // second softmax group (warps 16-19)
 constexpr int kKGroup0 = 5 * 32;  // first thread of the K warps
 constexpr int kVGroup0 = 9 * 32;  // first thread of the V warps
-constexpr uint32_t kBarSoftmax = 3, kBarCopy = 4;  // named barriers (128, 64 threads)
+constexpr uint32_t kBarSoftmax = 3, kBarCopy = 4;  // named barriers (256, 64 threads)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;
 constexpr int kMaxPolls = 1 << 22;
@@ -91,7 +94,7 @@ enum : int {
   kBarKEmpty = kBarVFull + kMaxSlots,  // [3] S MMAs that read the K tile done (commit)
   kBarVEmpty = kBarKEmpty + kMaxSlots, // [3] PV MMAs that read the V tile done (commit)
   kBarSFull = kBarVEmpty + kMaxSlots,  // [4] S chunk in TMEM (commit)
-  kBarPFull = kBarSFull + kMaxSBufs, // [4] P chunk in TMEM (128 arrivals)
+  kBarPFull = kBarSFull + kMaxSBufs, // [4] P chunk in TMEM (256 arrivals)
   kBarPFree = kBarPFull + kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
   kBarQReady = kBarPFree + kMaxSBufs,  // Q rows in TMEM (128 arrivals)
   kBarRawEmpty = kBarQReady + 1,  // [2][3] K, V raw stage read by every dequant thread (128 arrivals)
@@ -127,7 +130,9 @@ struct PrefillShape {
   static constexpr int kNumBars = kNumBarriers;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffIds = kOffMisc + 64;             // [kMaxIds] block ids
-  static constexpr int kBytes = kOffIds + kMaxIds * 4;
+  // softmax groups' exchange: chunk maxima [2 chunks][2 groups][128 rows], row sums [2][128]
+  static constexpr int kOffXchg = kOffIds + kMaxIds * 4;
+  static constexpr int kBytes = kOffXchg + (2 * 2 * kRows + 2 * kRows) * 4;
   static size_t smem_bytes() {
     const size_t need = (size_t)kBytes + 1024;  // + alignment of the base
     return need > kMinSmem ? need : kMinSmem;
@@ -422,10 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
 
   if (tid == 0) {
     for (int i = 0; i < S::kNumBars; ++i) {
-      const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) ||
-                        (i >= kBarPFull && i < kBarPFull + kMaxSBufs) || i == kBarQReady ||
+      const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) || i == kBarQReady ||
                         (i >= kBarRawEmpty && i < kBarRawEmpty + 2 * kMaxRawStages);
-      mbar_init(&bars[i], many ? 128u : (i == kBarFin ? 2u : 1u));
+      const bool pfull = i >= kBarPFull && i < kBarPFull + kMaxSBufs;
+      mbar_init(&bars[i], pfull ? 256u : many ? 128u : (i == kBarFin ? 2u : 1u));
     }
     misc->abort = 0;
     misc->softmax_stop[0] = misc->softmax_stop[1] = 0;
@@ -437,13 +442,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
   tc::fence_after_sync();
   const uint32_t tb = misc->tmem_base;
 
-  if (warp < 4) {
-    // ------------------------------------------------ Q, softmax, epilogue
-    const int r = tid;
+  if (warp < 4 || warp >= kSoftmax1Warp0) {
+    // ------------------------------------------------ Q, softmax, epilogue:
+    // two groups of 128 threads, thread (warp % 4, lane) of each on row
+    // r = TMEM lane 32 (warp % 4) + lane; group wg takes keys [wg CH/2,
+    // (wg + 1) CH/2) of every chunk and columns [wg D/2, (wg + 1) D/2) of O.
+    // They exchange chunk maxima (and at the end row sums) through shared
+    // memory, and both take every decision on the running max from the same
+    // values, so they agree on it.
+    const int wg = warp < 4 ? 0 : 1;
+    const int r = ((warp & 3) << 5) | lane;
     const int tok = r / G, g = r % G;
     const bool row_ok = (r < TQ * G) && (qtok0 + tok < q_len);
     const int pos = L - q_len + qtok0 + tok;  // absolute position (may be < 0: sees nothing)
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float* xmax = reinterpret_cast<float*>(base + S::kOffXchg);  // [2][2][kRows]
+    float* xsum = xmax + 4 * kRows;                                // [2][kRows]
     const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
                                 (long long)(q_begin + qtok0 + tok) * a.q_token_stride +
                                 (long long)(h * G + g) * D;
@@ -465,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     const float qmult = a.sm_scale * __ldg(a.kv_scales) * kLog2e *
                         __uint_as_float((uint32_t)(127 - sh) << 23);
 #pragma unroll 1
-    for (int blk = 0; blk < D / 64; ++blk) {
+    for (int blk = 0; wg == 0 && blk < D / 64; ++blk) {  // (group 0 writes Q)
       uint32_t w[32];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -479,39 +493,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       }
       tc::tmem_st32(tb + lane_off + S::kColQ + blk * 32, w);
     }
-    tc::tmem_wait_st();
-    tc::fence_before_sync();
-    tc::mbar_arrive(&bars[kBarQReady]);
+    if (wg == 0) {
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[kBarQReady]);
+    }
 
     float m_run = -INFINITY, l_run = 0.0f;
     volatile int* stop = misc->softmax_stop;
     int done_chunks = 0;
-    constexpr int CH = S::kChunk;
+    constexpr int CH = S::kChunk, HC = CH / 2;  // keys per chunk, per group
+    static_assert(HC == 32, "a group's half chunk is one 32-column TMEM load");
     for (int c = 0; c < nchunk; ++c) {
       const int sb = c % S::kSBufs;
       const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / S::kSBufs) & 1), misc, status, SM_WAIT);
       if (!ok) stop[c & 1] = 1;
-      tc::named_sync(kBarSoftmax, 128);
-      if (stop[c & 1]) break;
       tc::fence_after_sync();
-      const uint32_t scol = tb + lane_off + S::kColS + CH * sb;
-      const int key0 = c * CH;
+      const uint32_t scol = tb + lane_off + S::kColS + CH * sb + HC * wg;
+      const int key0 = c * CH + HC * wg;
       const int lim = min(pos + 1, kv_end) - key0;  // keys [key0, key0 + lim) are visible
-      // pass 1: max of the visible logits, in log2 units (32 columns at a time;
-      // the loops stay rolled to keep the hot code small)
+      // pass 1: max of the group's visible logits, in log2 units
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // (independent chains)
-#pragma unroll 1
-      for (int half = 0; half < CH / 32; ++half) {
+      {
         uint32_t sv[32];
-        tc::tmem_ld32(scol + 32 * half, sv);
+        tc::tmem_ld32(scol, sv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float x = (32 * half + i < lim) ? __uint_as_float(sv[i]) * qmult : -INFINITY;
+          const float x = (i < lim) ? __uint_as_float(sv[i]) * qmult : -INFINITY;
           mx4[i & 3] = fmaxf(mx4[i & 3], x);
         }
       }
-      const float cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float hmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      // (two exchange slots: a group writes slot c & 1 again only after both
+      // groups have passed the barrier of chunk c + 1)
+      xmax[((c & 1) * 2 + wg) * kRows + r] = hmax;
+      tc::named_sync(kBarSoftmax, 256);
+      if (stop[c & 1]) break;
+      const float cmax = fmaxf(hmax, xmax[((c & 1) * 2 + (wg ^ 1)) * kRows + r]);
       // lazy max: move it (and rescale O) only when this chunk exceeds it by > 2^8
       const bool up = (m_run == -INFINITY) ? (cmax > -INFINITY) : (cmax > m_run + kRescaleThresh);
       const bool need_o = up && m_run != -INFINITY;  // O holds earlier contributions
@@ -531,13 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         if (__all_sync(0xffffffffu, wok)) {
           tc::fence_after_sync();
 #pragma unroll 1
-          for (int blk = 0; blk < D / 16; ++blk) {
+          for (int blk = 0; blk < D / 32; ++blk) {  // the group's half of O
+            const uint32_t oc = tb + lane_off + S::kColO + wg * (D / 2) + blk * 16;
             uint32_t o[16];
-            tc::tmem_ld16(tb + lane_off + S::kColO + blk * 16, o);
+            tc::tmem_ld16(oc, o);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tc::tmem_st16(tb + lane_off + S::kColO + blk * 16, o);
+            tc::tmem_st16(oc, o);
           }
           tc::tmem_wait_st();
         } else {
@@ -550,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // no visible key yet: P = 0
       float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
-      for (int grp = 0; grp < CH / 16; ++grp) {
+      for (int grp = 0; grp < HC / 16; ++grp) {
         uint32_t sv[16], pw[16];
         tc::tmem_ld16(scol + 16 * grp, sv);
         tc::tmem_wait_ld();
@@ -584,6 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       have_o = __all_sync(0xffffffffu, ok);
     }
     tc::fence_after_sync();
+    // the row sum over both groups' keys (the same sum in both: a + b = b + a)
+    xsum[wg * kRows + r] = l_run;
+    tc::named_sync(kBarSoftmax, 256);
+    l_run += xsum[(wg ^ 1) * kRows + r];
     const float v_scale = __ldg(a.kv_scales + 1);
     const float o_scale = __ldg(a.o_scale);
     const float inv_os = 1.0f / o_scale;
@@ -594,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     const bool vec16 = (reinterpret_cast<uintptr_t>(a.o_bf16) & 15) == 0;
     const bool vec32 = (reinterpret_cast<uintptr_t>(a.o_f32) & 15) == 0;
 #pragma unroll 1
-    for (int blk = 0; blk < D / 32; ++blk) {
+    for (int blk = wg * (D / 64); blk < (wg + 1) * (D / 64); ++blk) {  // the group's half of O
       uint32_t o[32];
       if (have_o) {  // (warp-uniform: every lane loads its row)
         tc::tmem_ld32(tb + lane_off + S::kColO + blk * 32, o);
@@ -663,19 +687,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     // thread issued), and the two order through them: S_j is issued once PV_{j-NB}
     // (which read the P buffer S_j overwrites) has completed, PV_c once the
     // softmax has turned S_c into P_c.
-    if (lane == 0 && nchunk > 0) {
+    // The whole warp runs the loop (its waits made warp-uniform); one elected
+    // lane issues each MMA and commit.
+    if (nchunk > 0) {
       constexpr int CH = S::kChunk;
       constexpr int NB = S::kSBufs, NS = S::kSlots;
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, wait_bar(bar, parity, misc, status, MMA_WAIT));
+      };
       bool ok = true;
       if (warp == kSWarp) {
         constexpr uint32_t kIdescS = tc::idesc_f16(kRows, CH, false);
         const uint32_t kbase = smem_u32(base + S::kOffK);
-        ok = wait_bar(&bars[kBarQReady], 0u, misc, status);
+        ok = wait_all(&bars[kBarQReady], 0u);
         for (int j = 0; ok && j < nchunk; ++j) {
           const int sb = j % NB, slot = j % NS;
-          ok = wait_bar(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1), misc, status, MMA_WAIT);
-          if (ok && j >= NB)
-            ok = wait_bar(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1), misc, status, MMA_WAIT);
+          ok = wait_all(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1));
+          if (ok && j >= NB) ok = wait_all(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1));
           if (!ok) break;
           tc::fence_after_sync();
           const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
@@ -685,18 +713,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
             // start address advanced in 16-byte units (stays below 2^14 units)
             const uint64_t desc =
                 desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
-            tc::mma_ts(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+            tc::mma_ts_elect(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
           }
-          tc::commit(&bars[kBarKEmpty + slot]);
-          tc::commit(&bars[kBarSFull + sb]);
+          tc::commit_elect(&bars[kBarKEmpty + slot]);
+          tc::commit_elect(&bars[kBarSFull + sb]);
         }
       } else {
         constexpr uint32_t kIdescPV = tc::idesc_f16(kRows, D, true);
         const uint32_t vbase = smem_u32(base + S::kOffV);
         for (int c = 0; ok && c < nchunk; ++c) {
           const int pb = c % NB, slot = c % NS;
-          ok = wait_bar(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1), misc, status, MMA_WAIT);
-          if (ok) ok = wait_bar(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1), misc, status, MMA_WAIT);
+          ok = wait_all(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1));
+          if (ok) ok = wait_all(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1));
           if (!ok) break;
           tc::fence_after_sync();
           const uint64_t desc0 = tc::sw128_desc(vbase + slot * S::TILE, CH * 128, 1024);
@@ -704,24 +732,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
 #pragma unroll
           for (int i = 0; i < CH / 16; ++i) {  // P hi, then P lo, per 16 keys
             const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
-            tc::mma_ts(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
-            tc::mma_ts(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
+            tc::mma_ts_elect(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
+            tc::mma_ts_elect(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
           }
-          tc::commit(&bars[kBarVEmpty + slot]);
-          tc::commit(&bars[kBarPFree + pb]);
+          tc::commit_elect(&bars[kBarVEmpty + slot]);
+          tc::commit_elect(&bars[kBarPFree + pb]);
         }
       }
-      // every MMA this thread issued has completed: the final barrier counts
+      // every MMA this warp issued has completed: the final barrier counts
       // both issuers
-      tc::commit(&bars[kBarFin]);
-    }
-    if (warp == kMmaWarp && lane == 0 && nchunk > 0) {
-      // (TMEM is released by this warp below, after every MMA has completed)
-      for (int i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(&bars[kBarFin], 0u)) break;
+      tc::commit_elect(&bars[kBarFin]);
+      if (warp == kMmaWarp) {
+        // (TMEM is released by this warp below, after every MMA has completed)
+        for (int i = 0; i < kMaxPolls; ++i)
+          if (mbar_try_wait(&bars[kBarFin], 0u)) break;
+      }
     }
     __syncwarp();
-  } else if (warp >= kCopyWarp0) {
+  } else if (warp == kCopyWarp0 || warp == kCopyWarp0 + 1) {
     copy_role<D, BS, FMT>(a, warp - kCopyWarp0, b, h, nchunk, kv_end, base, bars, misc, status);
   } else {
     // K (warps 5-8) and V (warps 9-12) run one copy of the code
