@@ -543,35 +543,59 @@ __device__ __forceinline__ void pv_tile_fp8(uint32_t vt, const LaneOffsets& lo, 
 
 // One unit of T 16-token tiles in the stage at shared address sbase. MASK:
 // tile t holds valid[t] usable keys (0: skipped).
-template <int D, int BS, bool MASK, bool DUP, int FMT>
-__device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, const LaneOffsets& lo,
+// 16-token tiles per step of a unit's rolled tile loop: two keep the unit's
+// code small enough for the instruction cache and still overlap two tiles'
+// shared-memory loads and MMAs (measured against 1 and 4 per step)
+constexpr int kDecodeTilesPerStep = 2;
+
+template <int D, int BS, bool MASK, bool DUP, int FMT, int TBM>
+__device__ __forceinline__ void decode_unit(uint32_t sbase, int rem, int pmask, const LaneOffsets& lo,
                                             const uint32_t (&bq)[D / 16][2], float qmult,
                                             uint32_t lo_sel, float (&m_run)[2], float (&l_run)[2],
                                             float (&acc)[D / 16][4], int g8, int t4) {
   using S = DecodeShape<D, BS, FMT>;
   constexpr int T = S::T, NCH = S::NCH;
-  float s[T][4];
+  constexpr int TB = TBM < T ? TBM : T;
+  static_assert(T % TB == 0, "tiles per step divide the unit");
+  // TB tiles per step of a rolled loop (TB == T: the whole unit at once)
+#pragma unroll 1
+  for (int t0 = 0; t0 < T; t0 += TB) {
+  int valid[TB];
+  bool any = !MASK;
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
+  for (int tb = 0; tb < TB; ++tb) {
+    int v = 16;
+    if constexpr (MASK) {
+      const int t = t0 + tb;
+      v = min(16, rem - 16 * t);
+      if (v < 0 || !((pmask >> (16 * t / BS)) & 1)) v = 0;
+      any |= v > 0;
+    }
+    valid[tb] = v;
+  }
+  if (!any) continue;  // (warp-uniform)
+  float s[TB][4];
+#pragma unroll
+  for (int t = 0; t < TB; ++t) {
     s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.0f;
     if (!MASK || valid[t] > 0) {
       if constexpr (FMT == kFmtFp8)
-        qk_tile_fp8<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
+        qk_tile_fp8<D, MASK>(sbase + S::ktile(t0 + t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
       else
-        qk_tile<D, MASK>(sbase + S::ktile(t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
+        qk_tile<D, MASK>(sbase + S::ktile(t0 + t), lo, MASK ? valid[t] : 16, g8, bq, s[t]);
     } else {
       s[t][0] = s[t][1] = s[t][2] = s[t][3] = -INFINITY;
     }
   }
   // ---- online softmax (log2 units). x = s * qmult - m_run; the max moves only
   // when some x exceeds the threshold (or on the first keys of a column).
-  float x[T][4];
+  float x[TB][4];
   float mx0 = -INFINITY, mx1 = -INFINITY;
   {
     const float mu0 = (m_run[0] == -INFINITY) ? 0.f : m_run[0];
     const float mu1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < TB; ++t) {
       x[t][0] = fmaf(s[t][0], qmult, -mu0);
       x[t][1] = fmaf(s[t][1], qmult, -mu1);
       x[t][2] = fmaf(s[t][2], qmult, -mu0);
@@ -585,12 +609,12 @@ __device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, co
   if (__any_sync(0xffffffffu, up)) {
     float c0 = -INFINITY, c1 = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < TB; ++t) {
       c0 = fmaxf(c0, fmaxf(s[t][0], s[t][2]));
       c1 = fmaxf(c1, fmaxf(s[t][1], s[t][3]));
     }
-    const float t0 = warp_max_g(c0) * qmult, t1 = warp_max_g(c1) * qmult;
-    const float n0 = fmaxf(m_run[0], t0), n1 = fmaxf(m_run[1], t1);
+    const float m0 = warp_max_g(c0) * qmult, m1 = warp_max_g(c1) * qmult;
+    const float n0 = fmaxf(m_run[0], m0), n1 = fmaxf(m_run[1], m1);
     const float nu0 = (n0 == -INFINITY) ? 0.f : n0;
     const float nu1 = (n1 == -INFINITY) ? 0.f : n1;
     // ex2(-inf) = 0 clears a column seen for the first time (its acc and l are 0)
@@ -608,33 +632,34 @@ __device__ __forceinline__ void decode_unit(uint32_t sbase, const int* valid, co
       acc[c][3] *= al1;
     }
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < TB; ++t) {
       x[t][0] = fmaf(s[t][0], qmult, -nu0);
       x[t][1] = fmaf(s[t][1], qmult, -nu1);
       x[t][2] = fmaf(s[t][2], qmult, -nu0);
       x[t][3] = fmaf(s[t][3], qmult, -nu1);
     }
   }
-  float p[T][4];
+  float p[TB][4];
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
+  for (int t = 0; t < TB; ++t) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) p[t][i] = ex2(x[t][i]);
     l_run[0] += p[t][0] + p[t][2];
     l_run[1] += p[t][1] + p[t][3];
   }
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
+  for (int t = 0; t < TB; ++t) {
     if (!MASK || valid[t] > 0) {
       uint32_t bp[2], bpl[2];
       p_fragments<DUP>(p[t], lo_sel, bp, bpl);
       if constexpr (FMT == kFmtFp8)
-        pv_tile_fp8<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp,
-                                  bpl, acc);
+        pv_tile_fp8<D, MASK, DUP>(sbase + S::ktile(t0 + t) + S::VOFF, lo, MASK ? valid[t] : 16,
+                                  t4, bp, bpl, acc);
       else
-        pv_tile<D, MASK, DUP>(sbase + S::ktile(t) + S::VOFF, lo, MASK ? valid[t] : 16, t4, bp,
-                              bpl, acc);
+        pv_tile<D, MASK, DUP>(sbase + S::ktile(t0 + t) + S::VOFF, lo, MASK ? valid[t] : 16, t4,
+                              bp, bpl, acc);
     }
+  }
   }
 }
 
@@ -712,7 +737,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FMT>::kMaxWarps * 32, 1)
     decode_attention_kernel(const __grid_constant__ AttentionArgs a) {
   using S = DecodeShape<D, BS, FMT>;
   constexpr int kStages = S::kStages;
-  constexpr int PAGE = S::PAGE, NCH = S::NCH, U = S::U, UT = S::UT, T = S::T;
+  constexpr int PAGE = S::PAGE, NCH = S::NCH, U = S::U, UT = S::UT;
   constexpr int STAGE = S::STAGE;
   extern __shared__ __align__(128) uint8_t smem[];
   const int nw = blockDim.x >> 5;
@@ -1109,21 +1134,11 @@ __global__ void __launch_bounds__(DecodeCfg<D, FMT>::kMaxWarps * 32, 1)
           const int rem = L - u * UT;  // keys of this unit (clipped per tile below)
           const int pmask = okbits & 0xFF;  // pages copied
           if (rem >= UT && pmask == (1 << U) - 1) {
-            decode_unit<D, BS, false, DUP, FMT>(sbase, nullptr, lo, bq, qmult, lo_sel, m_run, l_run,
-                                           acc, g8, t4);
+            decode_unit<D, BS, false, DUP, FMT, kDecodeTilesPerStep>(
+                sbase, rem, pmask, lo, bq, qmult, lo_sel, m_run, l_run, acc, g8, t4);
           } else {
-            int vv[T];
-            bool any = false;
-#pragma unroll
-            for (int t = 0; t < T; ++t) {
-              int v = min(16, rem - 16 * t);
-              if (v < 0 || !((pmask >> (16 * t / BS)) & 1)) v = 0;
-              vv[t] = v;
-              any |= v > 0;
-            }
-            if (any)
-              decode_unit<D, BS, true, DUP, FMT>(sbase, vv, lo, bq, qmult, lo_sel, m_run, l_run, acc,
-                                            g8, t4);
+            decode_unit<D, BS, true, DUP, FMT, kDecodeTilesPerStep>(
+                sbase, rem, pmask, lo, bq, qmult, lo_sel, m_run, l_run, acc, g8, t4);
           }
           __syncwarp();
           if (!poisoned && k + kStages < nk) issue(k + kStages);

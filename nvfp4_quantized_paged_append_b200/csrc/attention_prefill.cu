@@ -94,8 +94,8 @@ enum : int {
   kBarKEmpty = kBarVFull + kMaxSlots,  // [3] S MMAs that read the K tile done (commit)
   kBarVEmpty = kBarKEmpty + kMaxSlots, // [3] PV MMAs that read the V tile done (commit)
   kBarSFull = kBarVEmpty + kMaxSlots,  // [4] S chunk in TMEM (commit)
-  kBarPFull = kBarSFull + kMaxSBufs, // [4] P chunk in TMEM (256 arrivals)
-  kBarPFree = kBarPFull + kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
+  kBarPFull = kBarSFull + kMaxSBufs, // [4][2] P of 16-key group g of both halves in TMEM (256 arrivals)
+  kBarPFree = kBarPFull + 2 * kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
   kBarQReady = kBarPFree + kMaxSBufs,  // Q rows in TMEM (128 arrivals)
   kBarRawEmpty = kBarQReady + 1,  // [2][3] K, V raw stage read by every dequant thread (128 arrivals)
   kBarFin = kBarRawEmpty + 2 * kMaxRawStages,  // every MMA issued done (2 commits)
@@ -130,9 +130,9 @@ struct PrefillShape {
   static constexpr int kNumBars = kNumBarriers;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffIds = kOffMisc + 64;             // [kMaxIds] block ids
-  // softmax groups' exchange: chunk maxima [2 chunks][2 groups][128 rows], row sums [2][128]
+  // the softmax groups' row sums [2 groups][128 rows]
   static constexpr int kOffXchg = kOffIds + kMaxIds * 4;
-  static constexpr int kBytes = kOffXchg + (2 * 2 * kRows + 2 * kRows) * 4;
+  static constexpr int kBytes = kOffXchg + 2 * kRows * 4;
   static size_t smem_bytes() {
     const size_t need = (size_t)kBytes + 1024;  // + alignment of the base
     return need > kMinSmem ? need : kMinSmem;
@@ -150,11 +150,6 @@ struct PrefillShape {
 struct Misc {
   uint32_t tmem_base;
   int abort;  // a wait of some role gave up: everyone stops
-  // the softmax group's stop flag, two alternating slots: chunk c's flag is
-  // written before the group's barrier of chunk c and read after it; the slot
-  // is written again only at chunk c + 2, after every thread of the group has
-  // passed the barrier of chunk c + 1
-  int softmax_stop[2];
   uint32_t raw_ok[2][kMaxRawStages];  // per raw stage: bit i = page i of the chunk was copied
 };
 
@@ -398,6 +393,27 @@ __device__ __forceinline__ void copy_role(const AttentionArgs& a, int kv, int b,
 
 }  // namespace
 
+// P of one 16-key group of a row: p = exp2(s * qmult - mu) (0 for keys at or
+// past glim when MASK), as f16 hi in pw[0..7] (keys in pairs) and
+// lo = f16(p - hi) in pw[8..15]; the p are added to ps4.
+template <bool MASK>
+__device__ __forceinline__ void p_group(const uint32_t (&sv)[16], float qmult, float mu, int glim,
+                                        uint32_t (&pw)[16], float (&ps4)[4]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), qmult, -mu));
+    float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), qmult, -mu));
+    if constexpr (MASK) {
+      p0 = (2 * i < glim) ? p0 : 0.0f;
+      p1 = (2 * i + 1 < glim) ? p1 : 0.0f;
+    }
+    ps4[i & 3] += p0 + p1;
+    pw[i] = pack_f16x2(p0, p1);
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
+    pw[8 + i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
+  }
+}
+
 template <int D, int BS, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const AttentionArgs a) {
   using S = PrefillShape<D, BS, FMT>;
@@ -429,11 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     for (int i = 0; i < S::kNumBars; ++i) {
       const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) || i == kBarQReady ||
                         (i >= kBarRawEmpty && i < kBarRawEmpty + 2 * kMaxRawStages);
-      const bool pfull = i >= kBarPFull && i < kBarPFull + kMaxSBufs;
+      const bool pfull = i >= kBarPFull && i < kBarPFull + 2 * kMaxSBufs;
       mbar_init(&bars[i], pfull ? 256u : many ? 128u : (i == kBarFin ? 2u : 1u));
     }
     misc->abort = 0;
-    misc->softmax_stop[0] = misc->softmax_stop[1] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tc::tmem_alloc(&misc->tmem_base, S::kTmemCols);
@@ -447,17 +462,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     // two groups of 128 threads, thread (warp % 4, lane) of each on row
     // r = TMEM lane 32 (warp % 4) + lane; group wg takes keys [wg CH/2,
     // (wg + 1) CH/2) of every chunk and columns [wg D/2, (wg + 1) D/2) of O.
-    // They exchange chunk maxima (and at the end row sums) through shared
-    // memory, and both take every decision on the running max from the same
-    // values, so they agree on it.
+    // Both compute each chunk's max over all its keys and take every decision
+    // on the running max from the same values, so they agree on it without
+    // exchanging anything; the row sums are added through shared memory at
+    // the end.
     const int wg = warp < 4 ? 0 : 1;
     const int r = ((warp & 3) << 5) | lane;
     const int tok = r / G, g = r % G;
     const bool row_ok = (r < TQ * G) && (qtok0 + tok < q_len);
     const int pos = L - q_len + qtok0 + tok;  // absolute position (may be < 0: sees nothing)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float* xmax = reinterpret_cast<float*>(base + S::kOffXchg);  // [2][2][kRows]
-    float* xsum = xmax + 4 * kRows;                                // [2][kRows]
+    float* xsum = reinterpret_cast<float*>(base + S::kOffXchg);  // [2][kRows]
     const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
                                 (long long)(q_begin + qtok0 + tok) * a.q_token_stride +
                                 (long long)(h * G + g) * D;
@@ -500,37 +515,50 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     }
 
     float m_run = -INFINITY, l_run = 0.0f;
-    volatile int* stop = misc->softmax_stop;
     int done_chunks = 0;
     constexpr int CH = S::kChunk, HC = CH / 2;  // keys per chunk, per group
     static_assert(HC == 32, "a group's half chunk is one 32-column TMEM load");
     for (int c = 0; c < nchunk; ++c) {
       const int sb = c % S::kSBufs;
       const bool ok = wait_bar(&bars[kBarSFull + sb], (uint32_t)((c / S::kSBufs) & 1), misc, status, SM_WAIT);
-      if (!ok) stop[c & 1] = 1;
+      if (!__all_sync(0xffffffffu, ok)) break;  // the block is aborting
       tc::fence_after_sync();
-      const uint32_t scol = tb + lane_off + S::kColS + CH * sb + HC * wg;
-      const int key0 = c * CH + HC * wg;
-      const int lim = min(pos + 1, kv_end) - key0;  // keys [key0, key0 + lim) are visible
-      // pass 1: max of the group's visible logits, in log2 units
+      const uint32_t ccol = tb + lane_off + S::kColS + CH * sb;  // the chunk's columns
+      const uint32_t scol = ccol + HC * wg;                      // this group's half
+      const int limc = min(pos + 1, kv_end) - c * CH;  // keys [c CH, c CH + limc) are visible
+      const int lim = limc - HC * wg;                  // the same, from this group's first key
+      // pass 1: max of the chunk's visible logits, in log2 units, over all CH
+      // keys (both groups compute it: no exchange). When every key of the
+      // chunk is visible to every row of the warp (all but the causal edge) and
+      // the scale is positive, the max of the raw logits is scaled once
+      // (rounding is monotone) and no key is masked.
+      const bool unmasked = __all_sync(0xffffffffu, limc >= CH && qmult > 0.0f);
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // (independent chains)
-      {
-        uint32_t sv[32];
-        tc::tmem_ld32(scol, sv);
-        tc::tmem_wait_ld();
+      float cmax;
+      if (unmasked) {
+#pragma unroll 1
+        for (int half = 0; half < CH / 32; ++half) {
+          uint32_t sv[32];
+          tc::tmem_ld32(ccol + 32 * half, sv);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = (i < lim) ? __uint_as_float(sv[i]) * qmult : -INFINITY;
-          mx4[i & 3] = fmaxf(mx4[i & 3], x);
+          for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(sv[i]));
         }
+        cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * qmult;
+      } else {
+#pragma unroll 1
+        for (int half = 0; half < CH / 32; ++half) {
+          uint32_t sv[32];
+          tc::tmem_ld32(ccol + 32 * half, sv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = (32 * half + i < limc) ? __uint_as_float(sv[i]) * qmult : -INFINITY;
+            mx4[i & 3] = fmaxf(mx4[i & 3], x);
+          }
+        }
+        cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       }
-      const float hmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      // (two exchange slots: a group writes slot c & 1 again only after both
-      // groups have passed the barrier of chunk c + 1)
-      xmax[((c & 1) * 2 + wg) * kRows + r] = hmax;
-      tc::named_sync(kBarSoftmax, 256);
-      if (stop[c & 1]) break;
-      const float cmax = fmaxf(hmax, xmax[((c & 1) * 2 + (wg ^ 1)) * kRows + r]);
       // lazy max: move it (and rescale O) only when this chunk exceeds it by > 2^8
       const bool up = (m_run == -INFINITY) ? (cmax > -INFINITY) : (cmax > m_run + kRescaleThresh);
       const bool need_o = up && m_run != -INFINITY;  // O holds earlier contributions
@@ -547,7 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         // done; that barrier is at most one phase behind here)
         bool wok = wait_bar(&bars[kBarPFree + (c - 1) % S::kSBufs], (uint32_t)(((c - 1) / S::kSBufs) & 1),
                             misc, status);
-        if (__all_sync(0xffffffffu, wok)) {
+        if (!__all_sync(0xffffffffu, wok)) break;  // the block is aborting
+        {
           tc::fence_after_sync();
 #pragma unroll 1
           for (int blk = 0; blk < D / 32; ++blk) {  // the group's half of O
@@ -560,8 +589,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
             tc::tmem_st16(oc, o);
           }
           tc::tmem_wait_st();
-        } else {
-          stop[(c + 1) & 1] = 1;  // read after the next chunk's barrier
         }
       }
       // pass 2: P = exp2(q.k * scale - m) per 16-key group, as f16 hi (8
@@ -574,23 +601,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         uint32_t sv[16], pw[16];
         tc::tmem_ld16(scol + 16 * grp, sv);
         tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int k0 = 16 * grp + 2 * i;
-          const float p0 = (k0 < lim) ? ex2(fmaf(__uint_as_float(sv[2 * i]), qmult, -mu)) : 0.0f;
-          const float p1 =
-              (k0 + 1 < lim) ? ex2(fmaf(__uint_as_float(sv[2 * i + 1]), qmult, -mu)) : 0.0f;
-          ps4[i & 3] += p0 + p1;
-          pw[i] = pack_f16x2(p0, p1);
-          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
-          pw[8 + i] = pack_f16x2(p0 - hf.x, p1 - hf.y);
-        }
+        if (unmasked)
+          p_group<false>(sv, qmult, mu, 0, pw, ps4);
+        else
+          p_group<true>(sv, qmult, mu, lim - 16 * grp, pw, ps4);
         tc::tmem_st16(scol + 16 * grp, pw);
+        // group grp of both halves ready: its PV MMAs may start while the
+        // next group is computed
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars[kBarPFull + 2 * sb + grp]);
       }
       l_run += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      tc::mbar_arrive(&bars[kBarPFull + sb]);
       done_chunks = c + 1;
     }
 
@@ -723,18 +745,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         const uint32_t vbase = smem_u32(base + S::kOffV);
         for (int c = 0; ok && c < nchunk; ++c) {
           const int pb = c % NB, slot = c % NS;
-          ok = wait_all(&bars[kBarPFull + pb], (uint32_t)((c / NB) & 1));
-          if (ok) ok = wait_all(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1));
-          if (!ok) break;
-          tc::fence_after_sync();
+          ok = wait_all(&bars[kBarVFull + slot], (uint32_t)((c / NS) & 1));
           const uint64_t desc0 = tc::sw128_desc(vbase + slot * S::TILE, CH * 128, 1024);
           const uint32_t pS = tb + S::kColS + CH * pb;
+          // 16-key group g of each half as soon as the softmax has written it:
+          // keys 16 g .. and CH/2 + 16 g .. (P hi, then P lo)
+#pragma unroll 1
+          for (int g = 0; ok && g < CH / 32; ++g) {
+            ok = wait_all(&bars[kBarPFull + 2 * pb + g], (uint32_t)((c / NB) & 1));
+            if (!ok) break;
+            tc::fence_after_sync();
 #pragma unroll
-          for (int i = 0; i < CH / 16; ++i) {  // P hi, then P lo, per 16 keys
-            const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
-            tc::mma_ts_elect(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
-            tc::mma_ts_elect(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
+            for (int hf = 0; hf < 2; ++hf) {
+              const int i = g + hf * (CH / 32);
+              const uint64_t desc = desc0 + (uint64_t)((i * 2048) >> 4);
+              tc::mma_ts_elect(tb + S::kColO, pS + i * 16, desc, kIdescPV, c > 0 || i > 0);
+              tc::mma_ts_elect(tb + S::kColO, pS + i * 16 + 8, desc, kIdescPV, true);
+            }
           }
+          if (!ok) break;
           tc::commit_elect(&bars[kBarVEmpty + slot]);
           tc::commit_elect(&bars[kBarPFree + pb]);
         }
