@@ -202,7 +202,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "decode_attention_kernel<128,16>": ["attention_decode.cu", "nvfp4kv_device.cuh",
                                         "nvfp4kv_launch.h"],
-    "quantize_append_kernel<128>": ["writer.cu", "nvfp4kv_device.cuh", "nvfp4kv_launch.h"],
+    "quantize_append_stream_kernel<128>": ["writer.cu", "nvfp4kv_device.cuh", "nvfp4kv_launch.h"],
 }
 
 
@@ -280,11 +280,30 @@ class DecodeState:
         nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
                            self.ws, o_bf16=self.o16, stream=stream, metadata_ready=metadata_ready)
 
-    def step(self, nk, stream=None, metadata_ready=False):
+    def step(self, nk, stream=None, metadata_ready=False, history_ready=False):
         """One decode step in one launch: append the new rows, attend."""
         nk.paged_decode_append(self.q, self.k_new, self.v_new, self.cache, self.bt, self.sl,
                                self.kvs, self.o8, self.osc, self.ws, o_bf16=self.o16,
-                               stream=stream, metadata_ready=metadata_ready)
+                               stream=stream, metadata_ready=metadata_ready,
+                               history_ready=history_ready)
+
+
+def cudart():
+    """The CUDA runtime library the process's torch uses (for per-step copies
+    and events without Python tensor overhead)."""
+    import ctypes
+    import glob
+    import torch
+    cands = glob.glob(os.path.join(os.path.dirname(torch.__file__), "lib", "libcudart.so*"))
+    try:
+        import nvidia.cuda_runtime as ncr
+        for d in ncr.__path__:
+            cands += glob.glob(os.path.join(d, "lib", "libcudart.so*"))
+    except ImportError:
+        pass
+    if not cands:
+        raise RuntimeError("libcudart not found next to torch")
+    return ctypes.CDLL(sorted(cands)[0])
 
 
 def build_cache(w, scales, dev):
@@ -557,13 +576,14 @@ def run_ours(args, rank, world, dist):
     # kernel alone.
     g_step, g_two, g_att = [], [], []
     # one round of steps (one per buffer copy) in one graph: each step's kernel is
-    # a programmatic dependent of the one before, so it starts reading its own
-    # metadata while that kernel finishes (it reads q and the cache only after
-    # that kernel has completed)
+    # a programmatic dependent of the one before, which writes neither its
+    # metadata nor its cache (another copy's), so it reads its metadata and
+    # starts its first page copies while that kernel finishes (q only after
+    # that kernel has completed), as after the projection kernel of a model
     g_round = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_round, stream=stream):
         for st in states:
-            st.step(nk, stream, metadata_ready=True)
+            st.step(nk, stream, history_ready=True)
     for st in states:
         ga = torch.cuda.CUDAGraph()
         with torch.cuda.graph(ga, stream=stream):
@@ -693,10 +713,33 @@ def run_ours(args, rank, world, dist):
                      st.k_new.stride(0), st.v_new.stride(0), p(st.cache), w.num_blocks,
                      w.block_size, H, D, p(st.bt), w.max_blocks_per_seq, p(st.sl), B,
                      p(st.kvs), ctypes.c_float(0.0), p(st.o8), p(st.osc), p(st.o16), None,
-                     p(st.ws), st.ws.numel(), 0, ctypes.c_void_p(stream.cuda_stream)))
-    h2d_done = [torch.cuda.Event() for _ in states]
-    step_done = [torch.cuda.Event() for _ in states]
-    d2h_done = [torch.cuda.Event() for _ in states]
+                     p(st.ws), st.ws.numel(),
+                     nk.NVFP4_ATTN_METADATA_READY | nk.NVFP4_ATTN_HISTORY_READY,
+                     ctypes.c_void_p(stream.cuda_stream)))
+    # the per-step copies and stream/event plumbing go straight to the CUDA
+    # runtime (a Python tensor copy or event costs more host time than the step)
+    rt = cudart()
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    rt.cudaMemcpyAsync.argtypes = [vp, vp, sz, ctypes.c_int, vp]
+    rt.cudaEventRecord.argtypes = [vp, vp]
+    rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+    rt.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+    rt.cudaEventDestroy.argtypes = [vp]
+
+    def new_event():
+        ev = vp()
+        if rt.cudaEventCreateWithFlags(ctypes.byref(ev), 2) != 0:  # timing disabled
+            raise RuntimeError("cudaEventCreateWithFlags failed")
+        return ev
+
+    h2d_done = [new_event() for _ in states]
+    step_done = [new_event() for _ in states]
+    d2h_done = [new_event() for _ in states]
+    s_up, s_down, s_main = (vp(x.cuda_stream) for x in (up_stream, down_stream, stream))
+    h_stage = vp(host_stage.data_ptr())
+    d_stage = [vp(st.stage.data_ptr()) for st in states]
+    h_out = [vp(t.data_ptr()) for t in host_outs]
+    d_out = [vp(st.o16.data_ptr()) for st in states]
     e2e_steps = max(50, min(500, args.steps))
     stream.synchronize()
     for it_ in range(e2e_steps + 10):
@@ -707,23 +750,23 @@ def run_ours(args, rank, world, dist):
             x0.record(stream)
         j = it_ % copies
         if it_ >= copies:  # the copy's previous result has left the device
-            up_stream.wait_event(d2h_done[j])
-        with torch.cuda.stream(up_stream):
-            states[j].stage.copy_(host_stage, non_blocking=True)
-        h2d_done[j].record(up_stream)
-        stream.wait_event(h2d_done[j])
+            rt.cudaStreamWaitEvent(s_up, d2h_done[j], 0)
+        rt.cudaMemcpyAsync(d_stage[j], h_stage, h2d, 1, s_up)
+        rt.cudaEventRecord(h2d_done[j], s_up)
+        rt.cudaStreamWaitEvent(s_main, h2d_done[j], 0)
         st_ = lib.nvfp4_paged_decode_append(*cargs[j])
         if st_ != 0:
             raise RuntimeError(f"nvfp4_paged_decode_append: {st_}")
-        step_done[j].record(stream)
-        down_stream.wait_event(step_done[j])
-        with torch.cuda.stream(down_stream):
-            host_outs[j].copy_(states[j].o16, non_blocking=True)
-        d2h_done[j].record(down_stream)
+        rt.cudaEventRecord(step_done[j], s_main)
+        rt.cudaStreamWaitEvent(s_down, step_done[j], 0)
+        rt.cudaMemcpyAsync(h_out[j], d_out[j], d2h, 2, s_down)
+        rt.cudaEventRecord(d2h_done[j], s_down)
     stream.wait_stream(down_stream)
     x1 = torch.cuda.Event(enable_timing=True)
     x1.record(stream)
     stream.synchronize()
+    for ev in h2d_done + step_done + d2h_done:
+        rt.cudaEventDestroy(ev)
     e2e_ms = max_over_ranks(x0.elapsed_time(x1) / e2e_steps, dist)
     del g_round, g_step, g_two, g_att, states
     torch.cuda.empty_cache()
@@ -786,7 +829,7 @@ def run_ours(args, rank, world, dist):
             "gbs": round(app_bytes / (app_ms * 1e-3) / 1e9, 1),
             "frac": round(app_bytes / (app_ms * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes": app_bytes,
-            "traffic": profiled_traffic("quantize_append_kernel<128>", "append_sweep"),
+            "traffic": profiled_traffic("quantize_append_stream_kernel<128>", "append_sweep"),
         },
         "long_decode": long_rec,
         "mixed_prefill_decode": mixed_rec,

@@ -173,8 +173,15 @@ NVFP4KV_API int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int
  * copied from the host before it); the kernel then reads them, builds its
  * work split, fetches block ids (setting NVFP4_DEV_BAD_BLOCK in the status
  * word for bad ones) before waiting, and reads q and the cache only after.
+ * With NVFP4_ATTN_HISTORY_READY (which implies NVFP4_ATTN_METADATA_READY) the
+ * caller further promises that the preceding kernel writes no cache page this
+ * call reads (for nvfp4_paged_decode_append: none of each sequence's keys
+ * before position seq_len - 1, the row the call writes itself), as when that
+ * kernel is the projection producing q; the first page copies then start
+ * before the wait as well, overlapping that kernel's tail.
  * flags = 0 is nvfp4_paged_attention. Unknown bits: NVFP4_ERR_INVALID_ARG. */
 #define NVFP4_ATTN_METADATA_READY 0x1u
+#define NVFP4_ATTN_HISTORY_READY 0x2u
 NVFP4KV_API int nvfp4_paged_attention_ex(
     const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
     const uint8_t* cache, int64_t num_blocks, int32_t block_size, int32_t num_kv_heads,

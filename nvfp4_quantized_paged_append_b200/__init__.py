@@ -30,6 +30,7 @@ DEV_BAD_BLOCK = 0x2
 DEV_TIMEOUT = 0x4
 DEV_BAD_QLEN = 0x8
 NVFP4_ATTN_METADATA_READY = 0x1
+NVFP4_ATTN_HISTORY_READY = 0x2
 
 
 class Nvfp4Error(RuntimeError):
@@ -252,12 +253,15 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                     sm_scale: float = 0.0, o_bf16: Optional[torch.Tensor] = None,
                     o_f32: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None,
-                    metadata_ready: bool = False, fp8: bool = False) -> None:
+                    metadata_ready: bool = False, fp8: bool = False,
+                    history_ready: bool = False) -> None:
     """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
     metadata_ready: the kernel launched just before on the stream writes none of
     block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
     attention kernel may read them while that kernel finishes
     (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it).
+    history_ready: that kernel writes no cache page either, so the first page
+    copies start early too (NVFP4_ATTN_HISTORY_READY; implies metadata_ready).
     fp8: the cache holds FP8-E4M3 rows (nvfp4_fp8kv_paged_attention)."""
     nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, qo_indptr,
                                                     o_fp8, o_bf16, o_f32, fp8)
@@ -267,8 +271,13 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
         _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(),
-        NVFP4_ATTN_METADATA_READY if metadata_ready else 0, _stream(stream))
+        _attn_flags(metadata_ready, history_ready), _stream(stream))
     _check(st, "nvfp4_paged_attention")
+
+
+def _attn_flags(metadata_ready: bool, history_ready: bool) -> int:
+    return (NVFP4_ATTN_METADATA_READY if metadata_ready else 0) | \
+        (NVFP4_ATTN_HISTORY_READY if history_ready else 0)
 
 
 def paged_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -278,10 +287,12 @@ def paged_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tenso
                         o_bf16: Optional[torch.Tensor] = None,
                         o_f32: Optional[torch.Tensor] = None,
                         stream: Optional[torch.cuda.Stream] = None,
-                        metadata_ready: bool = False) -> None:
+                        metadata_ready: bool = False, history_ready: bool = False) -> None:
     """One decode step in one launch: write every sequence's newest k/v row
     (position seq_lens[b] - 1) into the NVFP4 cache and run decode attention
-    over all keys. q [B, Hq, D], k_new / v_new [B, Hkv, D] bf16."""
+    over all keys. q [B, Hq, D], k_new / v_new [B, Hkv, D] bf16. metadata_ready
+    and history_ready as for paged_attention (history: the keys before
+    position seq_lens[b] - 1)."""
     nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, None,
                                                     o_fp8, o_bf16, o_f32)
     for name, x in (("k_new", k_new), ("v_new", v_new)):
@@ -295,7 +306,7 @@ def paged_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tenso
         _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb, _ptr(seq_lens), B, _ptr(kv_scales),
         float(sm_scale), _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(),
-        NVFP4_ATTN_METADATA_READY if metadata_ready else 0, _stream(stream))
+        _attn_flags(metadata_ready, history_ready), _stream(stream))
     _check(st, "nvfp4_paged_decode_append")
 
 

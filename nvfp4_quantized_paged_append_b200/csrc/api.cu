@@ -241,7 +241,8 @@ static int paged_attention_fmt(const void* q, int64_t q_token_stride, int64_t nu
                                void* o_bf16, float* o_f32, void* workspace,
                                size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream,
                                int kv_format) {
-  if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~(NVFP4_ATTN_METADATA_READY | NVFP4_ATTN_HISTORY_READY))
+    return NVFP4_ERR_INVALID_ARG;
   nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
       q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
       head_size, block_table, max_blocks_per_seq, seq_lens, qo_indptr, num_seqs, max_q_len,
@@ -327,7 +328,8 @@ int nvfp4_paged_decode_append(const void* q, int64_t q_token_stride, int32_t num
                               float sm_scale, uint8_t* o_fp8, const float* o_scale, void* o_bf16,
                               float* o_f32, void* workspace, size_t workspace_bytes,
                               uint32_t flags, nvfp4_stream_t stream) {
-  if (flags & ~NVFP4_ATTN_METADATA_READY) return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~(NVFP4_ATTN_METADATA_READY | NVFP4_ATTN_HISTORY_READY))
+    return NVFP4_ERR_INVALID_ARG;
   nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
       q, q_token_stride, num_seqs, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
       head_size, block_table, max_blocks_per_seq, seq_lens, nullptr, num_seqs, 1, kv_scales,

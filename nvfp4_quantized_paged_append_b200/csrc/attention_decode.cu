@@ -762,7 +762,10 @@ __global__ void __launch_bounds__(DecodeCfg<D, FMT>::kMaxWarps * 32, 1)
   // nothing that kernel may write before it has completed and its writes are
   // visible. With metadata_ready the batch metadata (sequence lengths, query
   // ranges, block table) is known not to be among them and is read first.
-  const bool metadata_ready = (a.flags & kAttnMetadataReady) != 0;
+  // With history_ready the history pages are not written by it either: the
+  // first page copies start before the wait too.
+  const bool history_ready = (a.flags & kAttnHistoryReady) != 0;
+  const bool metadata_ready = history_ready || (a.flags & kAttnMetadataReady) != 0;
   // The next kernel on the stream, if launched as a programmatic dependent,
   // may start its blocks on SMs this grid frees; like this one, it waits for
   // this grid's completion before reading anything this grid writes.
@@ -962,13 +965,16 @@ __global__ void __launch_bounds__(DecodeCfg<D, FMT>::kMaxWarps * 32, 1)
     };
 
     batch_load(0);
+    if (history_ready)
+      for (int k = 0; k < min(kStages, nk); ++k) issue(k);
     if (metadata_ready) grid_dependency_wait();  // q, cache and workspace from here on
     {
       int b, h, ss;
       locate(s, b, h, ss);
       fetch_q(b, h);
     }
-    for (int k = 0; k < min(kStages, nk); ++k) issue(k);
+    if (!history_ready)
+      for (int k = 0; k < min(kStages, nk); ++k) issue(k);
 
     const float k_scale = __ldg(a.kv_scales);
     const LaneOffsets lo = FMT == kFmtFp8 ? lane_offsets_fp8<D>(g8, t4) : lane_offsets<D>(g8, t4);

@@ -21,6 +21,7 @@ constexpr uint32_t kDevBadBlock = 0x2u;
 constexpr uint32_t kDevTimeout = 0x4u;
 constexpr uint32_t kDevBadQlen = 0x8u;
 constexpr uint32_t kAttnMetadataReady = 0x1u;  // NVFP4_ATTN_METADATA_READY
+constexpr uint32_t kAttnHistoryReady = 0x2u;   // NVFP4_ATTN_HISTORY_READY
 
 // Wait until the grids this one depends on (programmatic dependent launch)
 // have completed and their writes are visible; returns at once otherwise.

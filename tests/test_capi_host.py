@@ -151,7 +151,9 @@ def test_attention_flags_and_output_alignment(L):
     fake = ctypes.c_void_p(0x1000)
     full = dict(q=fake, cache=fake, bt=fake, sl=fake, kvs=fake, o8=fake, osc=fake)
     ready = nk.NVFP4_ATTN_METADATA_READY
-    assert _attn_ex(L, 0x2, **full) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, 0x4, **full) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, nk.NVFP4_ATTN_HISTORY_READY, B=0) == nk.NVFP4_OK
+    assert _attn_ex(L, nk.NVFP4_ATTN_HISTORY_READY | ready, **full) == nk.NVFP4_ERR_WORKSPACE
     assert _attn_ex(L, 0x80000000, B=0) == nk.NVFP4_ERR_INVALID_ARG
     assert _attn_ex(L, ready, B=0) == nk.NVFP4_OK
     assert _attn_ex(L, ready, **full) == nk.NVFP4_ERR_WORKSPACE      # same checks as flags = 0
@@ -212,7 +214,8 @@ def test_fused_decode_append_validation(L):
     assert call(v=None) == nk.NVFP4_ERR_INVALID_ARG
     assert call(ks=8 * 128 - 8) == nk.NVFP4_ERR_INVALID_ARG        # stride below a token row
     assert call(k=P(0x1008)) == nk.NVFP4_ERR_INVALID_ARG            # rows not 16-byte aligned
-    assert call(flags=0x2) == nk.NVFP4_ERR_INVALID_ARG
+    assert call(flags=0x4) == nk.NVFP4_ERR_INVALID_ARG
+    assert call(flags=0x3, B=0) == nk.NVFP4_OK                      # both known flags
     assert call(wsb=16) == nk.NVFP4_ERR_WORKSPACE
     assert call(d=96) == nk.NVFP4_ERR_UNSUPPORTED
     assert call(B=0) == nk.NVFP4_OK                                 # empty batch: nothing to do

@@ -131,3 +131,38 @@ def test_fused_decode_append_bad_block_flagged():
     diff = (cache != hist).nonzero()
     assert diff.numel() > 0
     assert set(diff[:, 0].tolist()) <= {int(x) for x in w.block_table[0, :3]}
+
+
+def test_fused_history_ready_chain():
+    """NVFP4_ATTN_HISTORY_READY: the step's first page copies start before it
+    waits for the preceding kernel. Chained after a step on another cache (the
+    flag's precondition), its cache and outputs equal those of the same step
+    launched with no flags, bit for bit."""
+    wa = wl.custom_workload("chain_a", 21, 16, 8, 128, 16, [300, 1200, 77, 2049],
+                            outliers="x20")
+    wb = wl.custom_workload("chain_b", 22, 16, 8, 128, 16, [900, 17, 3000, 640],
+                            outliers="x20")
+    runs = {}
+    for flags in ("plain", "history"):
+        outs = []
+        for w in (wa, wb):
+            scales = wl.global_scales(w, DEV)
+            hist, _, k_new, v_new = _history_cache(w, scales)
+            ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, DEV)
+            outs.append((w, scales, hist, k_new, v_new, ws, _outputs(w)))
+        torch.cuda.synchronize()
+        for i, (w, scales, cache, k_new, v_new, ws, (o8, o16, o32)) in enumerate(outs):
+            nk.paged_decode_append(wl.queries(w, DEV), k_new, v_new, cache,
+                                   torch.from_numpy(w.block_table).to(DEV),
+                                   torch.from_numpy(w.seq_lens).to(DEV),
+                                   torch.tensor([scales[0], scales[1]], device=DEV), o8,
+                                   dev_scalar(scales[2]), ws, o_bf16=o16, o_f32=o32,
+                                   history_ready=(flags == "history" and i == 1))
+        torch.cuda.synchronize()
+        for o in outs:
+            assert nk.read_device_status(o[5]) == (nk.NVFP4_OK, 0)
+        runs[flags] = [(o[2].clone(), [t.clone() for t in o[6]]) for o in outs]
+    for (ca, oa), (cb, ob) in zip(runs["plain"], runs["history"]):
+        assert torch.equal(ca, cb)
+        for x, y in zip(oa, ob):
+            assert torch.equal(x, y)
