@@ -55,6 +55,10 @@ def lib():
         _lib.nvo_paged_attention.restype = None
         _lib.nvo_paged_attention_fmt.argtypes = _lib.nvo_paged_attention.argtypes + [ctypes.c_int]
         _lib.nvo_paged_attention_fmt.restype = None
+        _lib.nvo_paged_attention_qfp4.argtypes = _lib.nvo_paged_attention.argtypes
+        _lib.nvo_paged_attention_qfp4.restype = None
+        _lib.nvo_q_row_global.argtypes = [P, ctypes.c_int]
+        _lib.nvo_q_row_global.restype = f32
         _lib.nvo_fp8kv_quantize_append_paged.argtypes = _lib.nvo_quantize_append_paged.argtypes
         _lib.nvo_fp8kv_quantize_append_paged.restype = i64
         _lib.nvo_act_sf_bytes.argtypes = [i64, i64, ctypes.c_int]
@@ -169,12 +173,14 @@ def fp8kv_quantize_append_paged(k, v, cache, slot_mapping, k_scale, v_scale, blo
 
 
 def paged_attention(q, cache, block_table, seq_lens, qo_indptr, k_scale,
-                    v_scale, sm_scale=0.0, o_scale=1.0, kv_format=KV_NVFP4):
+                    v_scale, sm_scale=0.0, o_scale=1.0, kv_format=KV_NVFP4, q_fp4=False):
     """fp64 paged attention. Returns (o_f64, o_fp8, o_bf16_bits).
 
     q: uint16 [Tq][Hq][D]; cache uint8[NB][2][Hkv][bs][F] (F = D/2 + D/16 for
     NVFP4, D for FP8 rows); block_table int32 [B][max_blocks]; seq_lens int32
-    [B]; qo_indptr int32 [B+1] or None.
+    [B]; qo_indptr int32 [B+1] or None. q_fp4 (NVFP4 cache only): the query
+    rows of sequences with more than one query are NVFP4-quantized first
+    (global scale per row, see q_row_global).
     """
     _need(q, np.uint16, "q")
     _need(cache, np.uint8, "cache")
@@ -188,11 +194,26 @@ def paged_attention(q, cache, block_table, seq_lens, qo_indptr, k_scale,
     o64 = np.zeros((tq, hq, d), np.float64)
     o8 = np.zeros((tq, hq, d), np.uint8)
     o16 = np.zeros((tq, hq, d), np.uint16)
-    lib().nvo_paged_attention_fmt(
-        _ptr(q), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
-        _ptr(seq_lens), _ptr(qo_indptr), B, k_scale, v_scale, sm_scale, o_scale,
-        _ptr(o64), _ptr(o8), _ptr(o16), int(kv_format))
+    if q_fp4:
+        if kv_format != KV_NVFP4:
+            raise ValueError("q_fp4 is defined over the NVFP4 cache")
+        lib().nvo_paged_attention_qfp4(
+            _ptr(q), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
+            _ptr(seq_lens), _ptr(qo_indptr), B, k_scale, v_scale, sm_scale, o_scale,
+            _ptr(o64), _ptr(o8), _ptr(o16))
+    else:
+        lib().nvo_paged_attention_fmt(
+            _ptr(q), tq, hq, _ptr(cache), nb, bs, hkv, d, _ptr(block_table), mb,
+            _ptr(seq_lens), _ptr(qo_indptr), B, k_scale, v_scale, sm_scale, o_scale,
+            _ptr(o64), _ptr(o8), _ptr(o16), int(kv_format))
     return o64, o8, o16
+
+
+def q_row_global(row) -> float:
+    """Global scale of an NVFP4-quantized query row (bf16 bits uint16[D]): the
+    smallest power of two g with amax / (6 g) <= 448 (1 for a zero row)."""
+    _need(row, np.uint16, "row")
+    return float(lib().nvo_q_row_global(_ptr(row), int(row.shape[-1])))
 
 
 # ---------------------------------------------------------------- activations

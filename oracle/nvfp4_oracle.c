@@ -286,15 +286,35 @@ void nvo_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
  * Outputs (each may be NULL): o_f64 [num_q_tokens][num_q_heads][head_size],
  * o_fp8 (E4M3 bytes), o_bf16 (bf16 bits), same shape.
  * Rows are independent; the loop over them is split across threads. */
-void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
-                             int num_q_heads, const uint8_t* cache,
-                             int64_t num_blocks, int block_size, int num_kv_heads,
-                             int head_size, const int32_t* block_table,
-                             int max_blocks_per_seq, const int32_t* seq_lens,
-                             const int32_t* qo_indptr, int num_seqs, float k_scale,
-                             float v_scale, double sm_scale, float o_scale,
-                             double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16,
-                             int kv_format) {
+/* NVFP4-Q variant (block-scaled QK^T): the global scale of a query
+ * row is the smallest power of two g with amax(row) / (6 g) <= 448, i.e.
+ * g = 2^ceil(log2(amax / 2688)) (1 for an all-zero row). Reading taken: the
+ * pages quantize activations with a per-tensor global scale but fix none for
+ * the query of a block-scaled QK^T; a per-row power of two keeps every block
+ * scale in E4M3's range and folds exactly into the logit scale. */
+float nvo_q_row_global(const uint16_t* x, int head_size) {
+  float amax = 0.0f;
+  for (int d = 0; d < head_size; ++d) {
+    float a = fabsf(nvo_bf16_to_f32(x[d]));
+    if (a > amax) amax = a;
+  }
+  if (!(amax > 0.0f)) return 1.0f;
+  int E;
+  frexpf(amax, &E);      /* amax in [2^(E-1), 2^E) */
+  int k = (E - 1) - 11;  /* 2688 = 1.3125 * 2^11: ceil(log2(amax/2688)) is k or k+1 */
+  if (ldexpf(2688.0f, k) >= amax) return ldexpf(1.0f, k);
+  return ldexpf(1.0f, k + 1);
+}
+
+static void attention_impl(const uint16_t* q, int64_t num_q_tokens,
+                           int num_q_heads, const uint8_t* cache,
+                           int64_t num_blocks, int block_size, int num_kv_heads,
+                           int head_size, const int32_t* block_table,
+                           int max_blocks_per_seq, const int32_t* seq_lens,
+                           const int32_t* qo_indptr, int num_seqs, float k_scale,
+                           float v_scale, double sm_scale, float o_scale,
+                           double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16,
+                           int kv_format, int q_fp4) {
   (void)num_blocks;
   (void)num_q_tokens;
   int64_t full_dim = kv_row_bytes(kv_format, head_size);
@@ -333,6 +353,20 @@ void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
     int64_t nkeys = last + 1 > 0 ? last + 1 : 0;
     if (nkeys > L) nkeys = L;
     const uint16_t* qrow = q + (tok * num_q_heads + hq) * (int64_t)head_size;
+    /* the query as the dot products see it: bf16, or (q_fp4, rows of
+     * sequences with more than one query) its NVFP4 round trip under the
+     * row's global scale */
+    double* qv = (double*)malloc(sizeof(double) * (size_t)head_size);
+    if (q_fp4 && q_len > 1) {
+      float g = nvo_q_row_global(qrow, head_size);
+      uint8_t* qq = (uint8_t*)malloc((size_t)(head_size / 2 + head_size / 16));
+      nvo_quantize_row(qrow, head_size, g, qq);
+      for (int d = 0; d < head_size; ++d)
+        qv[d] = row_elem(qq, head_size, d) * (double)g;
+      free(qq);
+    } else {
+      for (int d = 0; d < head_size; ++d) qv[d] = (double)nvo_bf16_to_f32(qrow[d]);
+    }
     double* z = (double*)malloc(sizeof(double) * (nkeys > 0 ? nkeys : 1));
     double* o = (double*)calloc((size_t)head_size, sizeof(double));
     double m = -INFINITY;
@@ -344,8 +378,7 @@ void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
                              block_size, full_dim);
       double dot = 0.0;
       for (int d = 0; d < head_size; ++d)
-        dot += (double)nvo_bf16_to_f32(qrow[d]) *
-               (kv_elem(kv_format, krow, head_size, d) * (double)k_scale);
+        dot += qv[d] * (kv_elem(kv_format, krow, head_size, d) * (double)k_scale);
       z[n] = sm_scale * dot;
       if (z[n] > m) m = z[n];
     }
@@ -373,9 +406,40 @@ void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
     }
     free(z);
     free(o);
+    free(qv);
   }
   free(row_seq);
   free(row_idx);
+}
+
+void nvo_paged_attention_fmt(const uint16_t* q, int64_t num_q_tokens,
+                             int num_q_heads, const uint8_t* cache,
+                             int64_t num_blocks, int block_size, int num_kv_heads,
+                             int head_size, const int32_t* block_table,
+                             int max_blocks_per_seq, const int32_t* seq_lens,
+                             const int32_t* qo_indptr, int num_seqs, float k_scale,
+                             float v_scale, double sm_scale, float o_scale,
+                             double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16,
+                             int kv_format) {
+  attention_impl(q, num_q_tokens, num_q_heads, cache, num_blocks, block_size,
+                 num_kv_heads, head_size, block_table, max_blocks_per_seq,
+                 seq_lens, qo_indptr, num_seqs, k_scale, v_scale, sm_scale,
+                 o_scale, o_f64, o_fp8, o_bf16, kv_format, 0);
+}
+
+/* NVFP4 cache, NVFP4-quantized queries in prefill rows (see nvo_q_row_global). */
+void nvo_paged_attention_qfp4(const uint16_t* q, int64_t num_q_tokens,
+                              int num_q_heads, const uint8_t* cache,
+                              int64_t num_blocks, int block_size, int num_kv_heads,
+                              int head_size, const int32_t* block_table,
+                              int max_blocks_per_seq, const int32_t* seq_lens,
+                              const int32_t* qo_indptr, int num_seqs, float k_scale,
+                              float v_scale, double sm_scale, float o_scale,
+                              double* o_f64, uint8_t* o_fp8, uint16_t* o_bf16) {
+  attention_impl(q, num_q_tokens, num_q_heads, cache, num_blocks, block_size,
+                 num_kv_heads, head_size, block_table, max_blocks_per_seq,
+                 seq_lens, qo_indptr, num_seqs, k_scale, v_scale, sm_scale,
+                 o_scale, o_f64, o_fp8, o_bf16, NVO_KV_NVFP4, 1);
 }
 
 /* NVFP4 cache (the format above). */

@@ -481,3 +481,97 @@ def test_fp8kv_attention_vs_dense_softmax():
                                        gk, gv, 0.0, 1.0, kv_format=oracle.KV_FP8)
     ref = _dense_attention(qd, xhat, table, seq_lens, q_lens, G, bs, gk, gv, 1 / math.sqrt(D))
     np.testing.assert_allclose(o64, ref, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------ NVFP4-quantized queries (block-scaled QK^T)
+@pytest.mark.parametrize("amax,g", [
+    (2688.0, 1.0),            # amax / (6 g) = 448 exactly
+    (2704.0, 2.0),            # just above: the next power of two
+    (1.0, 2.0 ** -11),        # 1 / (6 * 2^-11) = 341.3 <= 448; 2^-12 gives 682.7
+    (1.3125, 2.0 ** -11),     # = 2688 * 2^-11: the bound itself
+    (1.3203125, 2.0 ** -10),  # one bf16 step above it
+    (0.0, 1.0),               # all-zero row
+])
+def test_q_row_global_hand_worked(amax, g):
+    row = _bf16_bits(np.array([amax, -0.5 * amax] + [0.0] * 14, np.float32))
+    assert oracle.q_row_global(row) == g
+
+
+def _qfp4_case(rng, D, bs, G, q_lens, seq_lens):
+    Hkv = 2
+    need = sum(-(-L // bs) for L in seq_lens)
+    NB = need + 2
+    cache, _ = _hand_cache(rng, NB, Hkv, bs, D)
+    perm = rng.permutation(NB).astype(np.int32)
+    width = max(-(-L // bs) for L in seq_lens)
+    table = np.zeros((len(seq_lens), width), np.int32)
+    pos = 0
+    for b, L in enumerate(seq_lens):
+        nblk = -(-L // bs)
+        table[b, :nblk] = perm[pos:pos + nblk]
+        pos += nblk
+    indptr = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    return cache, table, np.array(seq_lens, np.int32), indptr, G * Hkv
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_qfp4_attention_is_attention_over_the_quantized_queries(D):
+    """Prefill rows: the NVFP4-Q attention equals plain attention over q-hat, the
+    queries round-tripped through the activation codec (pinned above) with
+    inv = 1 / g per row; q-hat (<= 6 significant bits) is exact in bf16. Decode
+    rows (one query) keep their bf16 query."""
+    rng = np.random.default_rng(90 + D)
+    q_lens, seq_lens = [3, 1, 5], [40, 33, 70]
+    cache, table, sl, indptr, Hq = _qfp4_case(rng, D, 16, 4, q_lens, seq_lens)
+    Tq = sum(q_lens)
+    q = _bf16_bits(rng.standard_normal((Tq, Hq, D)).astype(np.float32) * 0.7)
+    qhat = q.copy()
+    for b in range(len(q_lens)):
+        if q_lens[b] == 1:
+            continue
+        for t in range(indptr[b], indptr[b + 1]):
+            for h in range(Hq):
+                g = oracle.q_row_global(np.ascontiguousarray(q[t, h]))
+                fp4, sf = oracle.quantize_activation(np.ascontiguousarray(q[t, h][None]),
+                                                     1.0 / g, swizzled=False)
+                codes = np.empty(D, np.uint8)
+                codes[0::2] = fp4[0] & 0xF
+                codes[1::2] = fp4[0] >> 4
+                grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float64)
+                e2 = grid[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+                sc = torch.from_numpy(sf[0].copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+                vals = e2 * np.repeat(sc, 16) * g
+                qhat[t, h] = _bf16_bits(vals.astype(np.float32))
+                back = (qhat[t, h].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+                assert np.array_equal(back, vals)            # exact in bf16
+    gk, gv = float(np.float32(0.05)), float(np.float32(1.7))
+    got = oracle.paged_attention(q, cache, table, sl, indptr, gk, gv, 0.0, 0.5, q_fp4=True)
+    want = oracle.paged_attention(qhat, cache, table, sl, indptr, gk, gv, 0.0, 0.5)
+    for a, b in zip(got, want):
+        assert np.array_equal(a, b)
+    plain = oracle.paged_attention(q, cache, table, sl, indptr, gk, gv, 0.0, 0.5)
+    dec = indptr[1]  # the decode row of sequence 1
+    assert np.array_equal(got[0][dec], plain[0][dec])
+    assert not np.array_equal(got[0], plain[0])      # the prefill rows did change
+
+
+def test_qfp4_identity_on_representable_queries():
+    """Queries on the E2M1 grid times per-group powers of two (each group holding
+    a 6) are fixed points of the quantizer: the NVFP4-Q attention equals the plain
+    one exactly."""
+    rng = np.random.default_rng(17)
+    D = 256
+    q_lens, seq_lens = [4, 2], [50, 21]
+    cache, table, sl, indptr, Hq = _qfp4_case(rng, D, 16, 2, q_lens, seq_lens)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    Tq = sum(q_lens)
+    vals = grid[rng.integers(0, 8, (Tq, Hq, D))] * np.where(rng.random((Tq, Hq, D)) < 0.5, -1, 1)
+    vals = vals.astype(np.float32)
+    vals[..., ::16] = 6.0                                   # each group's amax is 6 * 2^j
+    vals *= np.repeat(2.0 ** (np.arange(D // 16) % 3), 16).astype(np.float32)
+    q = _bf16_bits(vals)
+    gk, gv = float(np.float32(0.05)), float(np.float32(1.7))
+    got = oracle.paged_attention(q, cache, table, sl, indptr, gk, gv, 0.0, 0.5, q_fp4=True)
+    want = oracle.paged_attention(q, cache, table, sl, indptr, gk, gv, 0.0, 0.5)
+    for a, b in zip(got, want):
+        assert np.array_equal(a, b)
