@@ -182,6 +182,15 @@ NVFP4KV_API int nvfp4_paged_attention(const void* q, int64_t q_token_stride, int
  * flags = 0 is nvfp4_paged_attention. Unknown bits: NVFP4_ERR_INVALID_ARG. */
 #define NVFP4_ATTN_METADATA_READY 0x1u
 #define NVFP4_ATTN_HISTORY_READY 0x2u
+/* NVFP4_ATTN_QFP4 (nvfp4_paged_attention_ex only; head size 256 over the NVFP4
+ * cache, else NVFP4_ERR_UNSUPPORTED): the rows of sequences with more than one
+ * query compute q K^T on the block-scaled tensor-core path
+ * (tcgen05 kind::mxf4nvf4), with each query row quantized to NVFP4 by the KV
+ * row codec under its own power-of-two global scale, the smallest g with
+ * max|q| / (6 g) <= 448, and K read as the cache's own codes and block scales.
+ * It changes the results (a variant measured against the same tolerance over
+ * the quantized queries); decode rows are unchanged. */
+#define NVFP4_ATTN_QFP4 0x4u
 NVFP4KV_API int nvfp4_paged_attention_ex(
     const void* q, int64_t q_token_stride, int64_t num_q_tokens, int32_t num_q_heads,
     const uint8_t* cache, int64_t num_blocks, int32_t block_size, int32_t num_kv_heads,

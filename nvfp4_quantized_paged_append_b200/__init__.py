@@ -31,6 +31,7 @@ DEV_TIMEOUT = 0x4
 DEV_BAD_QLEN = 0x8
 NVFP4_ATTN_METADATA_READY = 0x1
 NVFP4_ATTN_HISTORY_READY = 0x2
+NVFP4_ATTN_QFP4 = 0x4
 
 
 class Nvfp4Error(RuntimeError):
@@ -254,7 +255,7 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
                     o_f32: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None,
                     metadata_ready: bool = False, fp8: bool = False,
-                    history_ready: bool = False) -> None:
+                    history_ready: bool = False, q_fp4: bool = False) -> None:
     """Paged decode / chunked-prefill attention; writes o_fp8 (and o_bf16/o_f32).
     metadata_ready: the kernel launched just before on the stream writes none of
     block_table, seq_lens, qo_indptr, kv_scales, o_scale and workspace, so the
@@ -262,7 +263,9 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
     (NVFP4_ATTN_METADATA_READY; q and the cache are read only after it).
     history_ready: that kernel writes no cache page either, so the first page
     copies start early too (NVFP4_ATTN_HISTORY_READY; implies metadata_ready).
-    fp8: the cache holds FP8-E4M3 rows (nvfp4_fp8kv_paged_attention)."""
+    fp8: the cache holds FP8-E4M3 rows (nvfp4_fp8kv_paged_attention).
+    q_fp4: prefill rows compute q K^T on the block-scaled tensor-core path with
+    each query row quantized to NVFP4 (NVFP4_ATTN_QFP4; head size 256)."""
     nb, hkv, bs, d, tq, hq, B, mb = _attention_dims(q, cache, block_table, seq_lens, qo_indptr,
                                                     o_fp8, o_bf16, o_f32, fp8)
     fn = lib().nvfp4_fp8kv_paged_attention if fp8 else lib().nvfp4_paged_attention_ex
@@ -271,7 +274,8 @@ def paged_attention(q: torch.Tensor, cache: torch.Tensor, block_table: torch.Ten
         _ptr(seq_lens), _ptr(qo_indptr), B, max_q_len, _ptr(kv_scales), float(sm_scale),
         _ptr(o_fp8), _ptr(o_scale), _ptr(o_bf16), _ptr(o_f32), _ptr(workspace),
         workspace.numel() * workspace.element_size(),
-        _attn_flags(metadata_ready, history_ready), _stream(stream))
+        _attn_flags(metadata_ready, history_ready) | (NVFP4_ATTN_QFP4 if q_fp4 else 0),
+        _stream(stream))
     _check(st, "nvfp4_paged_attention")
 
 

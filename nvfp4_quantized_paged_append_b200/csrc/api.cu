@@ -241,8 +241,11 @@ static int paged_attention_fmt(const void* q, int64_t q_token_stride, int64_t nu
                                void* o_bf16, float* o_f32, void* workspace,
                                size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream,
                                int kv_format) {
-  if (flags & ~(NVFP4_ATTN_METADATA_READY | NVFP4_ATTN_HISTORY_READY))
+  if (flags & ~(NVFP4_ATTN_METADATA_READY | NVFP4_ATTN_HISTORY_READY | NVFP4_ATTN_QFP4))
     return NVFP4_ERR_INVALID_ARG;
+  // NVFP4 queries (block-scaled QK^T in prefill rows): head size 256, NVFP4 cache
+  if ((flags & NVFP4_ATTN_QFP4) && (head_size != 256 || kv_format != 0))
+    return NVFP4_ERR_UNSUPPORTED;
   nvfp4kv::AttentionArgs a = nvfp4kv::attention_args(
       q, q_token_stride, num_q_tokens, num_q_heads, cache, num_blocks, block_size, num_kv_heads,
       head_size, block_table, max_blocks_per_seq, seq_lens, qo_indptr, num_seqs, max_q_len,

@@ -98,18 +98,22 @@ enum : int {
   kBarPFree = kBarPFull + 2 * kMaxSBufs, // [4] PV MMAs that read a P buffer done (commit)
   kBarQReady = kBarPFree + kMaxSBufs,  // Q rows in TMEM (128 arrivals)
   kBarRawEmpty = kBarQReady + 1,  // [2][3] K, V raw stage read by every dequant thread (128 arrivals)
-  kBarFin = kBarRawEmpty + 2 * kMaxRawStages,  // every MMA issued done (2 commits)
+  kBarSRead = kBarRawEmpty + 2 * kMaxRawStages,  // [4] S chunk read by both softmax groups (256 arrivals)
+  kBarFin = kBarSRead + kMaxSBufs,  // every MMA issued done (2 commits)
   kNumBarriers = kBarFin + 1
 };
 
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 struct PrefillShape {
   // keys per chunk: N of S = Q K^T and the K-extent of O += P V. S/P buffers
   // in TMEM: four, or two at head size 256 (where O and Q take 384 of the 512
   // columns); f16 K and V tile slots: three, or two at head size 256 (shared
   // memory).
+  static_assert(!QF || (D == 256 && FMT == 0),
+                "NVFP4 queries: head size 256 over the NVFP4 cache");
   static constexpr int kChunk = 64;
-  static constexpr int kSBufs = D == 256 ? 2 : 4;
+  // (QF: Q leaves TMEM for shared memory, making room for a third buffer)
+  static constexpr int kSBufs = QF ? 3 : (D == 256 ? 2 : 4);
   static constexpr int kSlots = D == 256 ? 2 : 3;
   // raw page stages per K and V: three, or two for FP8 rows at head size 256
   static constexpr int kRawStages = (FMT && D == 256) ? 2 : 3;
@@ -118,15 +122,28 @@ struct PrefillShape {
   static constexpr int PPC = kChunk >= BS ? kChunk / BS : 1;  // pages per chunk
   static constexpr int RAW = kChunk * F;       // cache bytes of a chunk (K or V)
   static constexpr int TILE = kChunk * D * 2;  // f16 tile of a chunk
-  // TMEM columns: O [0, D), S/P buffers [D, D + 4 chunk), Q after them (D/2)
+  // QF: a K slot holds the chunk's E2M1 codes (K-major, 128B swizzle, one
+  // 128-byte row per key) and one 512-byte scale tile per K step of 64
+  static constexpr int KSTEPS = D / 64;
+  static constexpr int KCODES = kChunk * D / 2;
+  static constexpr int KTILE = QF ? KCODES + KSTEPS * 512 : TILE;
+  // QF: the Q tile, codes (128 rows x 128 bytes, swizzled as K) then its scale tiles
+  static constexpr int QCODES = kRows * D / 2;
+  static constexpr int QTILE = QF ? QCODES + KSTEPS * 512 : 0;
+  // TMEM columns: O [0, D), S/P buffers [D, D + kSBufs chunk), then Q (D/2, f16)
+  // or, QF, the scale factors: Q's (4 columns per K step), then each K slot's
   static constexpr uint32_t kColO = 0, kColS = D, kColQ = D + kSBufs * kChunk;
-  static constexpr uint32_t kTmemCols = (kColQ + D / 2 <= 256) ? 256u : 512u;
+  static constexpr uint32_t kColSFA = kColQ, kColSFB = kColSFA + 4 * KSTEPS;
+  static constexpr uint32_t kSFBSlot = 4 * KSTEPS;
+  static constexpr uint32_t kColEnd = QF ? kColSFB + kSlots * kSFBSlot : kColQ + D / 2;
+  static constexpr uint32_t kTmemCols = (kColEnd <= 256) ? 256u : 512u;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kSlots * TILE;
-  static constexpr int kOffKraw = 2 * kSlots * TILE;
+  static constexpr int kOffV = kSlots * KTILE;
+  static constexpr int kOffKraw = kOffV + kSlots * TILE;
   static constexpr int kOffVraw = kOffKraw + kRawStages * RAW;
-  static constexpr int kOffBar = kOffVraw + kRawStages * RAW;
+  static constexpr int kOffQ4 = kOffVraw + kRawStages * RAW;
+  static constexpr int kOffBar = kOffQ4 + QTILE;
   static constexpr int kNumBars = kNumBarriers;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffIds = kOffMisc + 64;             // [kMaxIds] block ids
@@ -139,7 +156,9 @@ struct PrefillShape {
   }
   static_assert(RAW % 16 == 0 && PAGE % 16 == 0, "bulk copies move 16-byte multiples");
   static_assert(TILE % 1024 == 0, "swizzle atoms sit on 1024-byte boundaries");
-  static_assert(kColQ + D / 2 <= 512, "TMEM budget");
+  static_assert(kColEnd <= 512, "TMEM budget");
+  static_assert(!QF || (KTILE % 1024 == 0 && kOffQ4 % 1024 == 0),
+                "swizzle atoms sit on 1024-byte boundaries");
   static_assert(kSBufs <= kMaxSBufs && kSlots <= kMaxSlots && kRawStages <= kMaxRawStages,
                 "barrier arrays");
   static_assert(kBytes + 1024 <= 227 * 1024, "shared memory per block");
@@ -189,11 +208,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* m
 // Issue the bulk copies of chunk c's pages (K: kv = 0, V: kv = 1) into raw
 // stage `st`; pages past kv_end or with a bad block id are not copied (the
 // latter flagged). One thread.
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 __device__ __forceinline__ void issue_chunk(const AttentionArgs& a, int b, int h, int kv, int c,
                                             int kv_end, uint8_t* raw, uint64_t* bar,
                                             uint32_t* ok_out, uint32_t* status, const int* ids) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   const int Hkv = a.num_kv_heads;
   uint32_t ok = 0, bytes = 0;
   long long src[S::PPC];
@@ -239,9 +258,9 @@ struct DequantPlan {
   int pg[2];         // their pages, within the chunk
 };
 
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 __device__ __forceinline__ DequantPlan dequant_plan(int gtid) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   static_assert(S::kChunk == 64, "the plan covers 64-key chunks with 4 warps");
   const int lane = gtid & 31, gw = gtid >> 5;
   const int n_lo = lane & 7, g_lo = lane >> 3;
@@ -260,10 +279,10 @@ __device__ __forceinline__ DequantPlan dequant_plan(int gtid) {
   return pl;
 }
 
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 __device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_t tile, int lim,
                                               const DequantPlan& pl) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   bool valid[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) valid[j] = (pl.n[j] < lim) && ((ok >> pl.pg[j]) & 1u);
@@ -315,13 +334,49 @@ __device__ __forceinline__ void dequant_chunk(uint32_t raw, uint32_t ok, uint32_
   }
 }
 
+// NVFP4 queries (QF): the K operand of S = Q K^T is the cache's own E2M1 codes
+// and E4M3 block scales, so a K chunk is repacked, not converted: each key's
+// D/2 code bytes become one 128-byte row of the slot's K-major tile (16-byte
+// chunk j stored at j ^ (key % 8)), and the key's 4 scales of K step t (one
+// 32-bit word of the raw row) go to byte offset (key % 32) * 16 + (key / 32) * 4
+// of the step's 512-byte scale tile: lane key % 32, column key / 32 once copied
+// to TMEM (the layout the block-scaled MMA reads its B scale factors in).
+// Keys at or past the visible end, and keys of pages not copied, get zero
+// codes and scales. 128 threads: thread i takes key i / 2, half i % 2 of its
+// row.
+template <int D, int BS, int FMT, bool QF>
+__device__ __forceinline__ void pack_chunk_k(uint32_t raw, uint32_t ok, uint32_t slot, int lim,
+                                             int gtid) {
+  using S = PrefillShape<D, BS, FMT, QF>;
+  const int n = gtid >> 1, hf = gtid & 1;
+  const bool valid = (n < lim) && ((ok >> (n / BS)) & 1u);
+  const uint32_t row = raw + (n / BS) * S::PAGE + (n % BS) * S::F;
+  const uint32_t dst = slot + (n >> 3) * 1024 + (n & 7) * 128;
+#pragma unroll
+  for (int jj = 0; jj < D / 64; ++jj) {  // this half's 16-byte code chunks
+    const int j = hf * (D / 64) + jj;
+    uint32_t w[4];
+    lds_v4(row + 16 * j, w);
+    uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
+    if (!valid) v = make_uint4(0u, 0u, 0u, 0u);
+    sts_v4(dst + ((j ^ (n & 7)) << 4), v);
+  }
+#pragma unroll
+  for (int tt = 0; tt < S::KSTEPS / 2; ++tt) {  // this half's K steps
+    const int t = hf * (S::KSTEPS / 2) + tt;
+    uint32_t sw = ld_shared_u32(row + D / 2 + 4 * t);
+    if (!valid) sw = 0u;
+    sts_u32(slot + S::KCODES + t * 512 + (n & 31) * 16 + (n >> 5) * 4, sw);
+  }
+}
+
 // Dequantization of one of K (kv = 0) and V (kv = 1), 128 threads: per chunk,
 // wait for its raw pages and a free tile slot, convert, and release both.
 // Every warp runs at its own pace (no barrier among the four).
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 __device__ __forceinline__ void dequant_role(int kv, int nchunk, int kv_end, uint8_t* base,
                                              uint64_t* bars, Misc* misc, uint32_t* status) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   const int gtid = threadIdx.x - (kv ? kVGroup0 : kKGroup0);
   const uint32_t raw_s = smem_u32(base + (kv ? S::kOffVraw : S::kOffKraw));
   const uint32_t tiles_s = smem_u32(base + (kv ? S::kOffV : S::kOffK));
@@ -330,15 +385,19 @@ __device__ __forceinline__ void dequant_role(int kv, int nchunk, int kv_end, uin
   uint64_t* full = bars + (kv ? kBarVFull : kBarKFull);
   uint64_t* empty = bars + (kv ? kBarVEmpty : kBarKEmpty);
   const volatile uint32_t* raw_ok = misc->raw_ok[kv];
-  const DequantPlan plan = dequant_plan<D, BS, FMT>(gtid);
+  const DequantPlan plan = dequant_plan<D, BS, FMT, QF>(gtid);
   for (int c = 0; c < nchunk; ++c) {
     const int st = c % S::kRawStages, slot = c % S::kSlots;
     bool ok = wait_bar(&raw_full[st], (uint32_t)((c / S::kRawStages) & 1), misc, status, KV_WAIT);
     if (ok && c >= S::kSlots)
       ok = wait_bar(&empty[slot], (uint32_t)((c / S::kSlots - 1) & 1), misc, status, KV_WAIT);
     if (!ok) break;  // the block is aborting
-    dequant_chunk<D, BS, FMT>(raw_s + st * S::RAW, raw_ok[st], tiles_s + slot * S::TILE,
-                              kv_end - c * S::kChunk, plan);
+    if (QF && kv == 0)
+      pack_chunk_k<D, BS, FMT, QF>(raw_s + st * S::RAW, raw_ok[st], tiles_s + slot * S::KTILE,
+                                   kv_end - c * S::kChunk, gtid);
+    else
+      dequant_chunk<D, BS, FMT, QF>(raw_s + st * S::RAW, raw_ok[st], tiles_s + slot * S::TILE,
+                                    kv_end - c * S::kChunk, plan);
     // generic-proxy writes of the tile (read by the tensor core) and reads of
     // the raw stage (next written by a bulk copy), both before the arrivals
     fence_proxy_async_smem();
@@ -352,11 +411,11 @@ __device__ __forceinline__ void dequant_role(int kv, int nchunk, int kv_end, uin
 // chunk that stage held. Both copy warps first stage the CTA's block ids in
 // shared memory (K and V pages share them). Before exit the thread waits for
 // every copy it issued to land (the copies write this CTA's shared memory).
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 __device__ __forceinline__ void copy_role(const AttentionArgs& a, int kv, int b, int h, int nchunk,
                                           int kv_end, uint8_t* base, uint64_t* bars, Misc* misc,
                                           uint32_t* status) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   const int lane = threadIdx.x & 31;
   uint8_t* raw = base + (kv ? S::kOffVraw : S::kOffKraw);
   uint64_t* raw_full = bars + (kv ? kBarVraw : kBarKraw);
@@ -378,7 +437,7 @@ __device__ __forceinline__ void copy_role(const AttentionArgs& a, int kv, int b,
         !wait_bar(&raw_empty[st], (uint32_t)((c / S::kRawStages - 1) & 1), misc, status,
                   kWaitSleep))
       break;
-    issue_chunk<D, BS, FMT>(a, b, h, kv, c, kv_end, raw + st * S::RAW, &raw_full[st], &raw_ok[st],
+    issue_chunk<D, BS, FMT, QF>(a, b, h, kv, c, kv_end, raw + st * S::RAW, &raw_full[st], &raw_ok[st],
                             status, ids);
     issued = c + 1;
   }
@@ -414,9 +473,21 @@ __device__ __forceinline__ void p_group(const uint32_t (&sv)[16], float qmult, f
   }
 }
 
-template <int D, int BS, int FMT>
+// Global scale of an NVFP4 query row with max |q| = amax: the smallest power
+// of two g with amax / (6 g) <= 448 (so no block scale saturates), 1 for a
+// zero row. With amax in [2^e, 2^(e+1)) and 2688 = 1.3125 * 2^11, that power is
+// 2^(e-11) or 2^(e-10).
+__device__ __forceinline__ float q_row_global(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  int E;
+  frexpf(amax, &E);  // amax in [2^(E-1), 2^E)
+  const int k = (E - 1) - 11;
+  return (ldexpf(2688.0f, k) >= amax) ? ldexpf(1.0f, k) : ldexpf(1.0f, k + 1);
+}
+
+template <int D, int BS, int FMT, bool QF>
 __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const AttentionArgs a) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -445,7 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     for (int i = 0; i < S::kNumBars; ++i) {
       const bool many = (i >= kBarKFull && i < kBarKFull + 2 * kMaxSlots) || i == kBarQReady ||
                         (i >= kBarRawEmpty && i < kBarRawEmpty + 2 * kMaxRawStages);
-      const bool pfull = i >= kBarPFull && i < kBarPFull + 2 * kMaxSBufs;
+      const bool pfull = (i >= kBarPFull && i < kBarPFull + 2 * kMaxSBufs) ||
+                         (i >= kBarSRead && i < kBarSRead + kMaxSBufs);
       mbar_init(&bars[i], pfull ? 256u : many ? 128u : (i == kBarFin ? 2u : 1u));
     }
     misc->abort = 0;
@@ -488,30 +560,72 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
                                fabsf(__uint_as_float(wv[j] & 0xFFFF0000u))));
       }
     }
-    const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
-    const int sh = min(126, max(-126, 15 - ex));
-    const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
-    const float qmult = a.sm_scale * __ldg(a.kv_scales) * kLog2e *
-                        __uint_as_float((uint32_t)(127 - sh) << 23);
+    float qmult;
+    if constexpr (QF) {
+      // NVFP4 queries: the row is quantized with the KV row codec under its
+      // global scale g (the smallest power of two with amax / (6 g) <= 448),
+      // codes into the Q tile (one 128-byte swizzled row per query row), the
+      // 4 scales of K step t into byte (r % 32) * 16 + (r / 32) * 4 of step t's
+      // scale tile; g joins the logit scale.
+      const float g = q_row_global(mx);
+      qmult = a.sm_scale * __ldg(a.kv_scales) * kLog2e * g;
+      if (wg == 0) {
+        const uint32_t q4 = smem_u32(base + S::kOffQ4);
+        const uint32_t qdst = q4 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll 1
-    for (int blk = 0; wg == 0 && blk < D / 64; ++blk) {  // (group 0 writes Q)
-      uint32_t w[32];
+        for (int t = 0; t < S::KSTEPS; ++t) {
+          uint32_t sw = 0u, cw[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
-        if (row_ok) v4 = __ldg(reinterpret_cast<const uint4*>(qrow + blk * 64) + j);
-        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+          for (int gi = 0; gi < 4; ++gi) {  // the step's 4 groups of 16
+            float x[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w[4 * j + i] = pack_f16x2(__uint_as_float(wv[i] << 16) * qs,
-                                    __uint_as_float(wv[i] & 0xFFFF0000u) * qs);
+            for (int j = 0; j < 2; ++j) {
+              uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+              if (row_ok) v4 = __ldg(reinterpret_cast<const uint4*>(qrow + t * 64 + gi * 16) + j);
+              const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                x[8 * j + 2 * i] = __uint_as_float(wv[i] << 16);
+                x[8 * j + 2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+              }
+            }
+            const uint32_t sb = quantize_group16(x, g, cw[2 * gi], cw[2 * gi + 1]);
+            sw |= sb << (8 * gi);
+          }
+          // the step's 32 code bytes: 16-byte chunks 2t and 2t + 1 of the row
+          sts_v4(qdst + (((2 * t) ^ (r & 7)) << 4), make_uint4(cw[0], cw[1], cw[2], cw[3]));
+          sts_v4(qdst + (((2 * t + 1) ^ (r & 7)) << 4), make_uint4(cw[4], cw[5], cw[6], cw[7]));
+          sts_u32(q4 + S::QCODES + t * 512 + (r & 31) * 16 + (r >> 5) * 4, sw);
+        }
+        fence_proxy_async_smem();  // read by the tensor core (MMA, scale copies)
+        tc::mbar_arrive(&bars[kBarQReady]);
       }
-      tc::tmem_st32(tb + lane_off + S::kColQ + blk * 32, w);
-    }
-    if (wg == 0) {
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      tc::mbar_arrive(&bars[kBarQReady]);
+    } else {
+      const int ex = (mx > 0.0f) ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 1;
+      const int sh = min(126, max(-126, 15 - ex));
+      const float qs = __uint_as_float((uint32_t)(sh + 127) << 23);
+      qmult = a.sm_scale * __ldg(a.kv_scales) * kLog2e *
+              __uint_as_float((uint32_t)(127 - sh) << 23);
+#pragma unroll 1
+      for (int blk = 0; wg == 0 && blk < D / 64; ++blk) {  // (group 0 writes Q)
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+          if (row_ok) v4 = __ldg(reinterpret_cast<const uint4*>(qrow + blk * 64) + j);
+          const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w[4 * j + i] = pack_f16x2(__uint_as_float(wv[i] << 16) * qs,
+                                      __uint_as_float(wv[i] & 0xFFFF0000u) * qs);
+        }
+        tc::tmem_st32(tb + lane_off + S::kColQ + blk * 32, w);
+      }
+      if (wg == 0) {
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars[kBarQReady]);
+      }
     }
 
     float m_run = -INFINITY, l_run = 0.0f;
@@ -559,6 +673,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         }
         cmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       }
+      // every logit of the chunk is in registers: the other group may now
+      // overwrite its half with P (it waits for this arrival before its first
+      // P store; so does this group)
+      tc::mbar_arrive(&bars[kBarSRead + sb]);
       // lazy max: move it (and rescale O) only when this chunk exceeds it by > 2^8
       const bool up = (m_run == -INFINITY) ? (cmax > -INFINITY) : (cmax > m_run + kRescaleThresh);
       const bool need_o = up && m_run != -INFINITY;  // O holds earlier contributions
@@ -595,6 +713,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       // columns, keys in pairs) and lo = f16(P - hi) (the next 8), written over
       // the group's own 16 logit columns (already read)
       const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // no visible key yet: P = 0
+      // both groups have read this chunk's logits (each reads all of them in
+      // pass 1) before either writes P over its half
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[kBarSRead + sb], (uint32_t)((c / S::kSBufs) & 1),
+                                            misc, status, SM_WAIT)))
+        break;
       float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
       for (int grp = 0; grp < HC / 16; ++grp) {
@@ -720,22 +843,50 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       bool ok = true;
       if (warp == kSWarp) {
         constexpr uint32_t kIdescS = tc::idesc_f16(kRows, CH, false);
+        constexpr uint32_t kIdescS4 = tc::idesc_mxf4nvf4(kRows, CH);
         const uint32_t kbase = smem_u32(base + S::kOffK);
+        const uint32_t q4 = smem_u32(base + S::kOffQ4);
         ok = wait_all(&bars[kBarQReady], 0u);
+        if (QF && ok) {
+          // Q's scale factors into TMEM once (the copies run before the MMAs
+          // this thread issues after them)
+          tc::fence_after_sync();
+#pragma unroll
+          for (int t = 0; t < S::KSTEPS; ++t)
+            tc::cp_32x128b_elect(tb + S::kColSFA + 4 * t, tc::plain_desc(q4 + S::QCODES + t * 512));
+        }
         for (int j = 0; ok && j < nchunk; ++j) {
           const int sb = j % NB, slot = j % NS;
           ok = wait_all(&bars[kBarKFull + slot], (uint32_t)((j / NS) & 1));
           if (ok && j >= NB) ok = wait_all(&bars[kBarPFree + sb], (uint32_t)((j / NB - 1) & 1));
           if (!ok) break;
           tc::fence_after_sync();
-          const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
           const uint32_t dS = tb + S::kColS + CH * sb;
+          if constexpr (QF) {
+            // block-scaled S = (Qc SFq)(Kc SFk)^T: K step t reads bytes
+            // [32 t, 32 t + 32) of every 128-byte row (start advanced in
+            // 16-byte units) and the step's scale columns
+            const uint32_t kt = kbase + slot * S::KTILE;
+            const uint32_t sfb = tb + S::kColSFB + slot * S::kSFBSlot;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // start address advanced in 16-byte units (stays below 2^14 units)
-            const uint64_t desc =
-                desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
-            tc::mma_ts_elect(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+            for (int t = 0; t < S::KSTEPS; ++t)
+              tc::cp_32x128b_elect(sfb + 4 * t, tc::plain_desc(kt + S::KCODES + t * 512));
+            const uint64_t adesc0 = tc::sw128_desc(q4, 16, 1024);
+            const uint64_t bdesc0 = tc::sw128_desc(kt, 16, 1024);
+#pragma unroll
+            for (int t = 0; t < S::KSTEPS; ++t)
+              tc::mma_mxf4_elect(dS, adesc0 + (uint64_t)((32 * t) >> 4),
+                                 bdesc0 + (uint64_t)((32 * t) >> 4), kIdescS4,
+                                 tb + S::kColSFA + 4 * t, sfb + 4 * t, t > 0);
+          } else {
+            const uint64_t desc0 = tc::sw128_desc(kbase + slot * S::TILE, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              // start address advanced in 16-byte units (stays below 2^14 units)
+              const uint64_t desc =
+                  desc0 + (uint64_t)(((kk >> 2) * (CH * 128) + (kk & 3) * 32) >> 4);
+              tc::mma_ts_elect(dS, tb + S::kColQ + kk * 8, desc, kIdescS, kk > 0);
+            }
           }
           tc::commit_elect(&bars[kBarKEmpty + slot]);
           tc::commit_elect(&bars[kBarSFull + sb]);
@@ -779,10 +930,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
     }
     __syncwarp();
   } else if (warp == kCopyWarp0 || warp == kCopyWarp0 + 1) {
-    copy_role<D, BS, FMT>(a, warp - kCopyWarp0, b, h, nchunk, kv_end, base, bars, misc, status);
+    copy_role<D, BS, FMT, QF>(a, warp - kCopyWarp0, b, h, nchunk, kv_end, base, bars, misc, status);
   } else {
     // K (warps 5-8) and V (warps 9-12) run one copy of the code
-    dequant_role<D, BS, FMT>(tid >= kVGroup0 ? 1 : 0, nchunk, kv_end, base, bars, misc, status);
+    dequant_role<D, BS, FMT, QF>(tid >= kVGroup0 ? 1 : 0, nchunk, kv_end, base, bars, misc, status);
   }
 
   tc::fence_before_sync();
@@ -793,11 +944,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
   }
 }
 
-template <int D, int BS, int FMT>
+template <int D, int BS, int FMT, bool QF>
 static cudaError_t launch_prefill_t(const AttentionArgs& a, cudaStream_t stream) {
-  using S = PrefillShape<D, BS, FMT>;
+  using S = PrefillShape<D, BS, FMT, QF>;
   const size_t smem = S::smem_bytes();
-  auto kern = prefill_attention_kernel<D, BS, FMT>;
+  auto kern = prefill_attention_kernel<D, BS, FMT, QF>;
   // the attribute is set once per (device, context), under a lock
   static std::mutex attr_mutex;
   static unsigned long long attr_ctx[64] = {0};
@@ -824,10 +975,15 @@ static cudaError_t launch_prefill_t(const AttentionArgs& a, cudaStream_t stream)
 }
 
 cudaError_t launch_prefill_attention(const AttentionArgs& a, cudaStream_t stream) {
+  if (a.flags & kAttnQfp4) {  // NVFP4 queries: head size 256, NVFP4 cache
+    if (a.head_size != 256 || a.kv_format != 0) return cudaErrorInvalidValue;
+    return a.block_size == 16 ? launch_prefill_t<256, 16, 0, true>(a, stream)
+                              : launch_prefill_t<256, 32, 0, true>(a, stream);
+  }
 #define NVFP4_PREFILL_CASE(DD, BB)                                             \
   if (a.head_size == DD && a.block_size == BB)                                 \
-    return a.kv_format ? launch_prefill_t<DD, BB, 1>(a, stream)                \
-                       : launch_prefill_t<DD, BB, 0>(a, stream);
+    return a.kv_format ? launch_prefill_t<DD, BB, 1, false>(a, stream)         \
+                       : launch_prefill_t<DD, BB, 0, false>(a, stream);
   NVFP4_PREFILL_CASE(64, 16)
   NVFP4_PREFILL_CASE(64, 32)
   NVFP4_PREFILL_CASE(128, 16)

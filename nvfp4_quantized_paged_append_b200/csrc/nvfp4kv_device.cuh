@@ -22,6 +22,7 @@ constexpr uint32_t kDevTimeout = 0x4u;
 constexpr uint32_t kDevBadQlen = 0x8u;
 constexpr uint32_t kAttnMetadataReady = 0x1u;  // NVFP4_ATTN_METADATA_READY
 constexpr uint32_t kAttnHistoryReady = 0x2u;   // NVFP4_ATTN_HISTORY_READY
+constexpr uint32_t kAttnQfp4 = 0x4u;           // NVFP4_ATTN_QFP4
 
 // Wait until the grids this one depends on (programmatic dependent launch)
 // have completed and their writes are visible; returns at once otherwise.
@@ -325,6 +326,9 @@ __device__ __forceinline__ uint32_t lds_b8(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u8 %0, [%1];\n" : "=r"(v) : "r"(addr));
   return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void sts_v4(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y),

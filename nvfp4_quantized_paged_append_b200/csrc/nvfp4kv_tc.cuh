@@ -104,6 +104,58 @@ __device__ __forceinline__ void commit_elect(uint64_t* bar) {
       : "memory");
 }
 
+// Shared-memory descriptor of a plain (unswizzled) K-major operand whose rows
+// are 16 bytes apart and whose 8-row core matrices are 128 bytes apart: the
+// source of a 32 x 128-bit tcgen05.cp.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 32;  // stride byte offset: next 8 rows
+  d |= (uint64_t)1 << 46;           // descriptor version
+  return d;                         // layout type 0: no swizzle
+}
+
+// Instruction descriptor of a block-scaled kind::mxf4nvf4 MMA: E2M1 A and B
+// (K-major), UE4M3 scale factors (one per 16 elements), fp32 accumulators,
+// M x N, K = 64 per instruction, scale factors at byte 0 of their columns.
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
+  return (1u << 7)                      // A format: E2M1
+         | (1u << 10)                   // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | (0u << 23)                   // scale format: UE4M3
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// D[tmem] (+)= (A * SFA) (B * SFB): A and B from shared memory (descriptors),
+// scale factors from TMEM; one elected lane of a converged warp issues.
+__device__ __forceinline__ void mma_mxf4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t sfa_tmem,
+                                               uint32_t sfb_tmem, bool accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p, e;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 rows x 128 bits from shared memory (plain_desc) into TMEM lanes 0-31 of 4
+// consecutive columns at taddr, replicated into all four lane quarters; one
+// elected lane of a converged warp issues (ordered with that thread's MMAs).
+__device__ __forceinline__ void cp_32x128b_elect(uint32_t taddr, uint64_t s_desc) {
+  asm volatile(
+      "{\n"
+      ".reg .pred e;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n"
+      "}\n" ::"r"(taddr),
+      "l"(s_desc)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every MMA this thread issued before has completed.
 __device__ __forceinline__ void commit(uint64_t* bar) {
   asm volatile(

@@ -151,7 +151,8 @@ def test_attention_flags_and_output_alignment(L):
     fake = ctypes.c_void_p(0x1000)
     full = dict(q=fake, cache=fake, bt=fake, sl=fake, kvs=fake, o8=fake, osc=fake)
     ready = nk.NVFP4_ATTN_METADATA_READY
-    assert _attn_ex(L, 0x4, **full) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, 0x8, **full) == nk.NVFP4_ERR_INVALID_ARG
+    assert _attn_ex(L, nk.NVFP4_ATTN_QFP4, **full) == nk.NVFP4_ERR_UNSUPPORTED  # head size 128
     assert _attn_ex(L, nk.NVFP4_ATTN_HISTORY_READY, B=0) == nk.NVFP4_OK
     assert _attn_ex(L, nk.NVFP4_ATTN_HISTORY_READY | ready, **full) == nk.NVFP4_ERR_WORKSPACE
     assert _attn_ex(L, 0x80000000, B=0) == nk.NVFP4_ERR_INVALID_ARG
