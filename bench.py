@@ -61,7 +61,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--profile", choices=["attention", "append", "step", "activation", "prefill"],
+    p.add_argument("--profile", choices=["attention", "append", "step", "activation", "prefill",
+                                          "prefill_qfp4"],
                    default=None,
                    help="kernel-only mode for profilers: set up, then launch the chosen "
                         "kernel --steps times (no timing, no JSON)")
@@ -338,10 +339,12 @@ class AttentionCall:
         self.o16 = torch.empty(shape, dtype=torch.bfloat16, device=dev)
         self.ws = nk.alloc_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_size, dev)
 
+    q_fp4 = False  # prefill rows on the block-scaled path with NVFP4 queries
+
     def __call__(self, stream):
         self.nk.paged_attention(self.q, self.cache, self.bt, self.sl, self.kvs, self.o8, self.osc,
                                 self.ws, qo_indptr=self.qo, max_q_len=self.w.max_q_len,
-                                o_bf16=self.o16, stream=stream)
+                                o_bf16=self.o16, stream=stream, q_fp4=self.q_fp4)
 
 
 def time_calls(fn, n, stream, warm=3):
@@ -412,6 +415,9 @@ def mixed_record(stream, clocks, region, n_prefill=5, n_decode=20):
     ms_full = time_calls(full, n_prefill, stream)
     ms_pre = time_calls(pre, n_prefill, stream)
     ms_dec = time_calls(dec, n_decode, stream)
+    pre.q_fp4 = True  # the same prefill with NVFP4 queries (block-scaled QK^T)
+    ms_pre4 = time_calls(pre, n_prefill, stream)
+    pre.q_fp4 = False
     clocks.mark()
     burst, sustained, tkind = tensor_peaks()
     peak, kind = peaks()
@@ -428,12 +434,18 @@ def mixed_record(stream, clocks, region, n_prefill=5, n_decode=20):
                        "frac": round(tf / sustained, 4),
                        "frac_of_burst": round(tf / burst, 4),
                        "prefill_kv_bytes": wp.kv_bytes()},
+           "prefill_qfp4": {"kernel": "the same prefill with NVFP4 queries (NVFP4_ATTN_QFP4: "
+                                      "q K^T on tcgen05 kind::mxf4nvf4; changes the results)",
+                            "ms": round(ms_pre4, 4),
+                            "tflops": round(flops / (ms_pre4 * 1e-3) / 1e12, 1),
+                            "frac": round(flops / (ms_pre4 * 1e-3) / 1e12 / sustained, 4)},
            "decode": {"kernel": "decode_attention_kernel<256,16>", "ms": round(ms_dec, 5),
                       "kv_bytes": wd.kv_bytes(), "gbs": round(dgbs, 1),
                       "frac": round(dgbs / peak, 4), "peak": peak,
                       "peak_kind": f"{kind} HBM copy"},
            "timing": f"back-to-back calls: {n_prefill} mixed, {n_prefill} prefill-only, "
-                     f"{n_decode} decode-only (CUDA events on the launching stream)",
+                     f"{n_decode} decode-only, {n_prefill} prefill-only with NVFP4 queries "
+                     f"(CUDA events on the launching stream)",
            "clocks": clocks.summary(region)}
     del cache, full, pre, dec
     torch.cuda.empty_cache()
@@ -973,7 +985,7 @@ def run_workload_times(args):
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
             nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, qo_indptr=qo,
-                               max_q_len=w.max_q_len)
+                               max_q_len=w.max_q_len, q_fp4=args.profile == "prefill_qfp4")
             e1.record()
             torch.cuda.synchronize()
             if i >= 2:
@@ -1037,7 +1049,7 @@ def run_profile(args):
         for _ in range(args.steps):
             nk.quantize_append_paged(k, v, cache, slots, ks, vs)
     else:
-        if args.profile == "prefill":
+        if args.profile in ("prefill", "prefill_qfp4"):
             # a small chunked-prefill batch with the mixed batch's shapes: 2
             # sequences of 512 causal queries over 2560 keys, 64 q / 8 kv heads,
             # head size 256, block size 16 (512 CTAs)

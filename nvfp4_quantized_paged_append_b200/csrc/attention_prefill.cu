@@ -114,7 +114,8 @@ struct PrefillShape {
   static constexpr int kChunk = 64;
   // (QF: Q leaves TMEM for shared memory, making room for a third buffer)
   static constexpr int kSBufs = QF ? 3 : (D == 256 ? 2 : 4);
-  static constexpr int kSlots = D == 256 ? 2 : 3;
+  // (QF: the K slots hold packed codes, 10 KB each, leaving room for three)
+  static constexpr int kSlots = (D == 256 && !QF) ? 2 : 3;
   // raw page stages per K and V: three, or two for FP8 rows at head size 256
   static constexpr int kRawStages = (FMT && D == 256) ? 2 : 3;
   static constexpr int F = FMT ? D : D / 2 + D / 16;  // row bytes: NVFP4, or FP8 (FMT = 1)
