@@ -985,7 +985,7 @@ def run_workload_times(args):
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
             nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, qo_indptr=qo,
-                               max_q_len=w.max_q_len, q_fp4=args.profile == "prefill_qfp4")
+                               max_q_len=w.max_q_len)
             e1.record()
             torch.cuda.synchronize()
             if i >= 2:
@@ -1076,7 +1076,7 @@ def run_profile(args):
         osc = torch.tensor([scales[2]], device=dev)
         for _ in range(args.steps):
             nk.paged_attention(q, cache, bt, sl, kvs, o8, osc, ws, qo_indptr=qo,
-                               max_q_len=w.max_q_len)
+                               max_q_len=w.max_q_len, q_fp4=args.profile == "prefill_qfp4")
     torch.cuda.synchronize()
     print(f"profile mode: {args.profile} x{args.steps} done", flush=True)
 
