@@ -714,12 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
       // columns, keys in pairs) and lo = f16(P - hi) (the next 8), written over
       // the group's own 16 logit columns (already read)
       const float mu = (m_run == -INFINITY) ? 0.0f : m_run;  // no visible key yet: P = 0
-      // both groups have read this chunk's logits (each reads all of them in
-      // pass 1) before either writes P over its half
-      if (!__all_sync(0xffffffffu, wait_bar(&bars[kBarSRead + sb], (uint32_t)((c / S::kSBufs) & 1),
-                                            misc, status, SM_WAIT)))
-        break;
       float ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      bool aborted = false;
 #pragma unroll 1
       for (int grp = 0; grp < HC / 16; ++grp) {
         uint32_t sv[16], pw[16];
@@ -729,6 +725,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
           p_group<false>(sv, qmult, mu, 0, pw, ps4);
         else
           p_group<true>(sv, qmult, mu, lim - 16 * grp, pw, ps4);
+        // both groups have read this chunk's logits (each reads all of them
+        // in pass 1) before either writes P over its half; the first group's
+        // P is computed before the wait, so skew between the groups hides
+        // behind it
+        if (grp == 0 &&
+            !__all_sync(0xffffffffu, wait_bar(&bars[kBarSRead + sb], (uint32_t)((c / S::kSBufs) & 1),
+                                              misc, status, SM_WAIT))) {
+          aborted = true;  // the block is aborting
+          break;
+        }
         tc::tmem_st16(scol + 16 * grp, pw);
         // group grp of both halves ready: its PV MMAs may start while the
         // next group is computed
@@ -736,6 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attention_kernel(const At
         tc::fence_before_sync();
         tc::mbar_arrive(&bars[kBarPFull + 2 * sb + grp]);
       }
+      if (aborted) break;
       l_run += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
       done_chunks = c + 1;
     }
