@@ -112,16 +112,47 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 }
 
 // ------------------------------------------------------------ NVFP4 encode
+// Packed fp32 pairs (Blackwell mul.rn.f32x2: two correctly rounded fp32
+// products per instruction; the low half is the first element).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+
+__device__ __forceinline__ void unpack_f32x2(uint64_t d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// max(a, b, c) in one instruction; a NaN operand is ignored like fmaxf's.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// The bracket around an approximate quotient: 1 -+ 2^-20.
+constexpr float kBracketLo = 0.99999904632568359375f;
+constexpr float kBracketHi = 1.00000095367431640625f;
+
 // E2M1 codes of fl32(x_i / S) for 8 values (element 2j in the low nibble of
-// byte j). Fast path: y = x * rcp.approx(S) is within 2^-21 (relative) of
-// x / S (the reciprocal is within 1 ulp, the product rounds by half an ulp),
-// and so is fl32(x / S). If y * (1 - 2^-20) and y * (1 + 2^-20) give the same
-// code, no rounding threshold of the E2M1 grid lies between them, and the
-// conversion is monotone, so fl32(x / S) has that code as well. Otherwise
-// (x / S within ~1e-6 of a threshold, exact ties included) the quotient is
-// formed with IEEE division. S must be a positive normal number; above
-// 2^100 the reciprocal nears the subnormal range, where its 1-ulp bound no
-// longer holds, so such scales always divide.
+// byte j). Fast path: with r = rcp.approx(S) (within 1 ulp of 1/S) and
+// r_lo = fl32(r (1 - 2^-20)), r_hi = fl32(r (1 + 2^-20)), the products
+// fl32(x r_lo) and fl32(x r_hi) lie strictly on either side of fl32(x / S)
+// (the errors of the reciprocal and the two roundings add up to less than
+// 2^-21, while the bracket is 2^-20 wide on each side). If both ends give the
+// same code, no rounding threshold of the E2M1 grid lies between them, and
+// the conversion is monotone, so fl32(x / S) has that code as well.
+// Otherwise (x / S within ~1e-6 of a threshold, exact ties included) the
+// quotient is formed with IEEE division. S must be a positive normal number;
+// above 2^100 the reciprocal nears the subnormal range, where its 1-ulp bound
+// no longer holds, so such scales always divide.
 __device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S) {
   if (S > 1.2676506e30f) {
     float q[8];
@@ -131,12 +162,15 @@ __device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S)
   }
   float r;
   asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(S));
+  const uint64_t rr = pack_f32x2(r, r);
+  const uint64_t r_lo = mul_f32x2(rr, pack_f32x2(kBracketLo, kBracketLo));
+  const uint64_t r_hi = mul_f32x2(rr, pack_f32x2(kBracketHi, kBracketHi));
   float lo[8], hi[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float y = x[i] * r;
-    lo[i] = y * 0.99999904632568359375f;  // 1 - 2^-20
-    hi[i] = y * 1.00000095367431640625f;  // 1 + 2^-20
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t p = pack_f32x2(x[2 * i], x[2 * i + 1]);
+    unpack_f32x2(mul_f32x2(p, r_lo), lo[2 * i], lo[2 * i + 1]);
+    unpack_f32x2(mul_f32x2(p, r_hi), hi[2 * i], hi[2 * i + 1]);
   }
   const uint32_t c_lo = f32x8_to_e2m1x8(lo);
   const uint32_t c_hi = f32x8_to_e2m1x8(hi);
@@ -148,16 +182,18 @@ __device__ __forceinline__ uint32_t e2m1_codes_div(const float (&x)[8], float S)
 }
 
 // E4M3 byte of fl32(a / b) (RNE, satfinite). Fast path as for the codes: the
-// quotient from the approximate reciprocal is within 2^-21 of fl32(a / b);
-// when both ends of the +-2^-20 bracket encode to the same byte, so does
-// fl32(a / b). Otherwise, and for b outside [2^-100, 2^100] or a non-finite
-// a, the quotient is formed with IEEE division.
+// bracketed products a r_lo and a r_hi (one packed multiply) lie on either
+// side of fl32(a / b); when both encode to the same byte, so does fl32(a / b).
+// Otherwise, and for b outside [2^-100, 2^100] or a non-finite a, the
+// quotient is formed with IEEE division.
 __device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float b) {
   if (b >= 7.8886091e-31f && b <= 1.2676506e30f && a <= 3.4028235e38f) {
     float r;
     asm("rcp.approx.f32 %0, %1;\n" : "=f"(r) : "f"(b));
-    const float y = a * r;
-    const uint32_t two = f32x2_to_e4m3x2(y * 0.99999904632568359375f, y * 1.00000095367431640625f);
+    const uint64_t rb = mul_f32x2(pack_f32x2(r, r), pack_f32x2(kBracketLo, kBracketHi));
+    float lo, hi;
+    unpack_f32x2(mul_f32x2(pack_f32x2(a, a), rb), lo, hi);
+    const uint32_t two = f32x2_to_e4m3x2(lo, hi);
     if ((two & 0xFFu) == (two >> 8)) return two & 0xFFu;
   }
   return f32_to_e4m3(__fdiv_rn(a, b));
@@ -168,11 +204,15 @@ __device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float b) {
 // block scale sb = E4M3(fl32(amax / fl32(6 g))) (returned) and the E2M1 codes
 // of fl32(x_i / fl32(E4M3(sb) g)) in c0 (elements 0..7) and c1 (8..15); every
 // code is 0 when that effective scale is 0. Bit-exact with IEEE fp32 division.
+// amax is the largest |x_i| with NaNs ignored (0 when all are NaN).
 __device__ __forceinline__ uint32_t quantize_group16(const float (&x)[16], float g, uint32_t& c0,
                                                      uint32_t& c1) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const float m0 = max3f(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]));
+  const float m1 = max3f(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+  const float m2 = max3f(fabsf(x[6]), fabsf(x[7]), fabsf(x[8]));
+  const float m3 = max3f(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
+  const float m4 = max3f(fabsf(x[12]), fabsf(x[13]), fabsf(x[14]));
+  const float amax = max3f(max3f(m0, m1, m2), max3f(m3, m4, fabsf(x[15])), 0.0f);
   const uint32_t sb = e4m3_of_quotient(amax, __fmul_rn(6.0f, g));
   const float S = __fmul_rn(e4m3_to_f32(sb), g);
   c0 = 0u;

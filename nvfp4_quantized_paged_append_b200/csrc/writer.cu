@@ -9,8 +9,10 @@
 // Dequant: "FlashInfer NVFP4 KV serving on pre-SM100 GPUs", quick answer (the
 // paged NVFP4 dequantize helper).
 //
-// Mapping: one CTA per token, one thread per 16-element block of a row (two
-// 16-byte bf16 loads, one E4M3 scale byte, 8 bytes of packed codes).
+// Mapping: grid-stride blocks over tokens, one thread per two adjacent
+// 16-element blocks of a row (NVFP4 rows of head size 128 or 256 when the
+// token's row groups come in multiples of 64), else one thread per 16-element
+// block; one CTA per token when a token has more groups than a block holds.
 #include <algorithm>
 
 #include "nvfp4kv_device.cuh"
@@ -159,6 +161,88 @@ __global__ void __launch_bounds__(1024) quantize_append_stream_kernel(
   }
 }
 
+// Grid-stride NVFP4 writer with two adjacent 16-element groups of a row per
+// thread (blockDim.x == num_kv_heads * D / 16; D = 128 or 256, whose rows
+// start on 8-byte boundaries): four 16-byte bf16 loads, 16
+// bytes of packed codes and a 2-byte pair of scales per token, so the token's
+// slot, address and loop work is shared by two groups. Same slot rules and
+// next-token prefetch as quantize_append_stream_kernel.
+template <int D>
+__global__ void __launch_bounds__(512) quantize_append_pair_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    int64_t k_stride, int64_t v_stride, int num_kv_heads, uint8_t* __restrict__ cache,
+    int64_t num_tokens, int64_t num_blocks, int bs_log2, const int64_t* __restrict__ slot_mapping,
+    const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+    uint32_t* __restrict__ status) {
+  constexpr int TPR = D / 32;  // threads per row
+  constexpr int F = D / 2 + D / 16;
+  static_assert(F % 8 == 0, "rows must be 8-byte aligned (head size 128 or 256)");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  const int idx = threadIdx.x;
+  const int rr = idx / TPR, j = idx % TPR;
+  const int kv = rr >= num_kv_heads ? 1 : 0;
+  const int h = rr - kv * num_kv_heads;
+  const __nv_bfloat16* src0 = (kv == 0 ? k : v) + h * D + j * 32;
+  const int64_t stride = kv == 0 ? k_stride : v_stride;
+  const float g = __ldg(kv == 0 ? k_scale : v_scale);
+  const int block_size = 1 << bs_log2;
+  int64_t t = blockIdx.x;
+  int64_t slot = -1;
+  uint4 r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (t < num_tokens) {
+    slot = __ldg(slot_mapping + t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __ldg(reinterpret_cast<const uint4*>(src0 + t * stride) + i);
+  }
+  while (t < num_tokens) {
+    const int64_t tn = t + gridDim.x;
+    int64_t slot_n = -1;
+    uint4 n[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) n[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tn < num_tokens) {
+      slot_n = __ldg(slot_mapping + tn);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) n[i] = __ldg(reinterpret_cast<const uint4*>(src0 + tn * stride) + i);
+    }
+    if (slot >= (num_blocks << bs_log2)) {
+      if (idx == 0 && status) atomicOr(status, kDevBadSlot);
+    } else if (slot >= 0) {
+      const int64_t blk = slot >> bs_log2;
+      const int off = (int)(slot & (block_size - 1));
+      uint8_t* dst =
+          cache + (((blk * 2 + kv) * num_kv_heads + h) * (int64_t)block_size + off) * F;
+      uint32_t cw[4], sbv[2];
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const uint32_t wv[8] = {r[2 * gi].x,     r[2 * gi].y,     r[2 * gi].z,     r[2 * gi].w,
+                                r[2 * gi + 1].x, r[2 * gi + 1].y, r[2 * gi + 1].z, r[2 * gi + 1].w};
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[2 * i] = __uint_as_float(wv[i] << 16);
+          x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        sbv[gi] = quantize_group16(x, g, cw[2 * gi], cw[2 * gi + 1]);
+      }
+      if constexpr (F % 16 == 0) {
+        *reinterpret_cast<uint4*>(dst + 16 * j) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      } else {  // rows 8-byte aligned
+        reinterpret_cast<uint2*>(dst + 16 * j)[0] = make_uint2(cw[0], cw[1]);
+        reinterpret_cast<uint2*>(dst + 16 * j)[1] = make_uint2(cw[2], cw[3]);
+      }
+      // D / 2 + 2 j and F are even: the scale pair is 2-byte aligned
+      *reinterpret_cast<uint16_t*>(dst + D / 2 + 2 * j) = (uint16_t)(sbv[0] | (sbv[1] << 8));
+    }
+    t = tn;
+    slot = slot_n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = n[i];
+  }
+}
+
 // FP8-E4M3 rows (the comparison format): code = E4M3 RNE satfinite of
 // fl32(x / g) per element (same bracketed reciprocal fast path, IEEE division
 // near rounding thresholds), D bytes per row in the same HND page layout.
@@ -246,14 +330,45 @@ cudaError_t launch_quantize_append(const QuantizeAppendArgs& a, cudaStream_t str
   const int rows_threads = 2 * a.num_kv_heads * (a.head_size / 16);
   const auto* k = static_cast<const __nv_bfloat16*>(a.k);
   const auto* v = static_cast<const __nv_bfloat16*>(a.v);
+  int dev = 0, sms = 0;
   if (rows_threads % 32 == 0 && rows_threads <= 1024) {
-    // grid-stride blocks, as many as are resident at once (tokens per block
-    // rise with the batch)
-    int dev = 0, sms = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (err != cudaSuccess) return err;
+  }
+  if (!a.kv_format && a.head_size >= 128 && rows_threads % 64 == 0 && rows_threads <= 1024) {
+    // NVFP4 rows of 8-byte aligned length, two groups per thread: grid-stride
+    // blocks, as many as are resident at once
+    const int threads = rows_threads / 2;
+    cudaError_t err = cudaSuccess;
+#define NVFP4_PAIR_CASE(DD)                                                                    \
+  case DD: {                                                                                   \
+    auto kern = quantize_append_pair_kernel<DD>;                                               \
+    int per_sm = 1;                                                                            \
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);            \
+    if (err != cudaSuccess) return err;                                                        \
+    const long long resident = (long long)sms * std::max(1, per_sm);                           \
+    const unsigned grid = (unsigned)std::min<long long>(a.num_tokens, resident);               \
+    kern<<<grid, threads, 0, stream>>>(k, v, a.k_token_stride, a.v_token_stride,               \
+                                       a.num_kv_heads, a.cache, a.num_tokens, a.num_blocks,    \
+                                       bs_log2, a.slot_mapping, a.k_scale, a.v_scale,          \
+                                       a.device_status);                                       \
+    break;                                                                                     \
+  }
+    switch (a.head_size) {
+      NVFP4_PAIR_CASE(128)
+      NVFP4_PAIR_CASE(256)
+      default:
+        return cudaErrorInvalidValue;
+    }
+#undef NVFP4_PAIR_CASE
+    return cudaGetLastError();
+  }
+  if (rows_threads % 32 == 0 && rows_threads <= 1024) {
+    // grid-stride blocks, as many as are resident at once (tokens per block
+    // rise with the batch)
+    cudaError_t err = cudaSuccess;
 #define NVFP4_STREAM_CASE(DD)                                                                  \
   case DD: {                                                                                   \
     auto kern = a.kv_format ? quantize_append_stream_kernel<DD, true>                          \

@@ -93,6 +93,28 @@ def test_codec_bruteforce_bit_exact(D, g):
     assert bad.size == 0, f"{len(bad)} bytes differ, first at {bad[:3].tolist()}"
 
 
+@pytest.mark.parametrize("D,H", [(64, 1), (64, 8), (128, 2), (128, 4), (256, 2), (256, 8)])
+@pytest.mark.parametrize("g", [0.37, 2.0 ** 110, 2.0 ** -120])
+def test_codec_bruteforce_every_writer_mapping(D, H, g):
+    """The same codec cases through each writer mapping: one CTA per token
+    (D 64, H 1), one thread per 16-element group (D 64 H 8, D 128 H 2), two
+    groups per thread (D 128 H 4, D 256 H 2 / 8); global scales that send the
+    effective scale above 2^100 (IEEE-division path) or make 6 g and the
+    scales subnormal."""
+    rng = np.random.default_rng(D * 13 + H)
+    T, bs = 256, 16
+    x = _codec_cases(rng, T, H, D) * np.float32(g)
+    k = _bf16(x)
+    v = _bf16(-x[::-1].copy())
+    nb = T // bs + 2
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    slots[rng.random(T) < 0.05] = -1
+    got = _gpu_write(k, v, slots, nb, bs, g, g * 0.75)
+    want = _oracle_write(k, v, slots, nb, bs, g, g * 0.75)
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, f"{len(bad)} bytes differ, first at {bad[:3].tolist()}"
+
+
 @pytest.mark.parametrize("name", ["tiny_decode", "qwen3_0p6b_decode"])
 def test_writer_decode_workloads_full(name):
     w = wl.make_workload(name)
