@@ -286,7 +286,8 @@ void nvo_dequantize_paged(const uint8_t* cache, int64_t num_blocks,
  * Outputs (each may be NULL): o_f64 [num_q_tokens][num_q_heads][head_size],
  * o_fp8 (E4M3 bytes), o_bf16 (bf16 bits), same shape.
  * Rows are independent; the loop over them is split across threads. */
-/* NVFP4-Q variant (block-scaled QK^T): the global scale of a query
+/* NVFP4 queries for a block-scaled QK^T (operand format of "Move NVFP4 GEMM
+ * management into NvFp4LinearKernel", base.py): the global scale of a query
  * row is the smallest power of two g with amax(row) / (6 g) <= 448, i.e.
  * g = 2^ceil(log2(amax / 2688)) (1 for an all-zero row). Reading taken: the
  * pages quantize activations with a per-tensor global scale but fix none for
